@@ -1,0 +1,154 @@
+"""fp64 CPU oracle for shifted local-window self-attention (test infrastructure).
+
+Only the test suite, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` /
+``--impl reference`` legs of ``bench.py`` may import this package.  The product
+path (``shifted_window_attention_swattn_b200``) never imports it and shares no
+code with it.
+
+The arithmetic lives in ``ref_swattn.c`` (plain C, fp64, one materialised array
+per stage).  This module only builds that file with gcc and marshals arguments
+through ctypes.  Method: "Backend-Agnostic Sparse Attention for Fast
+High-Resolution Visual Generation" (BASA), §3.1 "Shifted Window Sparse
+Attention" and Appendix A.1 "Regular execution with standard attention
+backends".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "ref_swattn.c")
+_LIB_PATH = os.path.join(_HERE, "libref_swattn.so")
+_lib = None
+_lock = threading.Lock()
+
+_I3 = ctypes.c_int * 3
+
+
+def build(force: bool = False) -> str:
+    """Compile ref_swattn.c into libref_swattn.so next to it (gcc, -O2)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c99", "-D_POSIX_C_SOURCE=200809L", "-Wall", "-fPIC", "-shared",
+             "-pthread", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            lib.oref_index_map.argtypes = [ctypes.c_int] * 3 + [_I3, _I3, ctypes.c_void_p, ctypes.c_void_p]
+            lib.oref_index_map.restype = ctypes.c_int
+            lib.oref_swattn_fwd.argtypes = (
+                [ctypes.c_void_p] * 4 + [ctypes.c_int] * 6 + [_I3, _I3, ctypes.c_double]
+                + [ctypes.c_int] * 3)
+            lib.oref_swattn_fwd.restype = ctypes.c_int
+            lib.oref_swattn_rows.argtypes = (
+                [ctypes.c_void_p] * 3 + [ctypes.c_int] * 6 + [_I3, _I3, ctypes.c_double]
+                + [ctypes.c_void_p, ctypes.c_long, ctypes.c_void_p])
+            lib.oref_swattn_rows.restype = ctypes.c_int
+            lib.oref_flops.argtypes = [ctypes.c_int] * 6 + [_I3]
+            lib.oref_flops.restype = ctypes.c_double
+            _lib = lib
+    return _lib
+
+
+def _bits(x) -> np.ndarray:
+    """bf16 data as a contiguous uint16 numpy array of bit patterns.
+
+    Accepts a torch bf16 tensor (any device) or a uint16 numpy array.
+    """
+    if isinstance(x, np.ndarray):
+        if x.dtype != np.uint16:
+            raise TypeError("numpy input must hold bf16 bit patterns as uint16")
+        return np.ascontiguousarray(x)
+    import torch  # local: the oracle itself needs only numpy
+    if x.dtype != torch.bfloat16:
+        raise TypeError("torch input must be bfloat16")
+    return x.detach().to("cpu").contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def _geom_args(win, shift):
+    if len(win) != 3 or len(shift) != 3:
+        raise ValueError("win and shift are (t, h, w) triples")
+    return _I3(*[int(a) for a in win]), _I3(*[int(a) for a in shift])
+
+
+def n_windows(T, H, W, win) -> int:
+    """Windows in the grid: ceil(n_a / w_a) per axis (truncated last windows)."""
+    n = 1
+    for ext, w in zip((T, H, W), win):
+        if int(w) < 1 or int(ext) < 1:
+            raise ValueError("grid and window extents must be >= 1")
+        n *= -(-int(ext) // int(w))
+    return n
+
+
+def index_map(T, H, W, win, shift):
+    """(token_of_slot [n_windows, w_t*w_h*w_w] int32 with -1 padding, count [n_windows])."""
+    lib = _load()
+    nw = n_windows(T, H, W, win)
+    nmax = int(win[0]) * int(win[1]) * int(win[2])
+    tos = np.empty((nw, nmax), dtype=np.int32)
+    cnt = np.empty((nw,), dtype=np.int32)
+    w3, s3 = _geom_args(win, shift)
+    rc = lib.oref_index_map(int(T), int(H), int(W), w3, s3, tos.ctypes.data, cnt.ctypes.data)
+    if rc != 0:
+        raise ValueError(f"oref_index_map failed ({rc})")
+    return tos, cnt
+
+
+def swattn_fwd(q, k, v, B, heads, T, H, W, d, win, shift, scale, head_range=None, nthreads=None):
+    """fp64 output [B, T*H*W, heads, d] of the shifted-window forward.
+
+    Heads outside ``head_range`` (default: all) are left as NaN.
+    """
+    lib = _load()
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    N = int(T) * int(H) * int(W)
+    expect = int(B) * N * int(heads) * int(d)
+    for a in (qb, kb, vb):
+        if a.size != expect:
+            raise ValueError("q/k/v must hold B*T*H*W*heads*d elements")
+    h0, h1 = (0, int(heads)) if head_range is None else (int(head_range[0]), int(head_range[1]))
+    if nthreads is None:
+        nthreads = max(1, len(os.sched_getaffinity(0)))
+    out = np.full((int(B), N, int(heads), int(d)), np.nan, dtype=np.float64)
+    w3, s3 = _geom_args(win, shift)
+    rc = lib.oref_swattn_fwd(qb.ctypes.data, kb.ctypes.data, vb.ctypes.data, out.ctypes.data,
+                             int(B), int(heads), int(T), int(H), int(W), int(d), w3, s3,
+                             float(scale), h0, h1, int(nthreads))
+    if rc != 0:
+        raise ValueError(f"oref_swattn_fwd failed ({rc})")
+    return out
+
+
+def swattn_rows(q, k, v, B, heads, T, H, W, d, win, shift, scale, triples):
+    """fp64 output rows [len(triples), d] for (b, token, head) triples."""
+    lib = _load()
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    tr = np.ascontiguousarray(np.asarray(triples, dtype=np.int64).reshape(-1, 3))
+    out = np.empty((tr.shape[0], int(d)), dtype=np.float64)
+    w3, s3 = _geom_args(win, shift)
+    rc = lib.oref_swattn_rows(qb.ctypes.data, kb.ctypes.data, vb.ctypes.data,
+                              int(B), int(heads), int(T), int(H), int(W), int(d), w3, s3,
+                              float(scale), tr.ctypes.data, tr.shape[0], out.ctypes.data)
+    if rc != 0:
+        raise ValueError(f"oref_swattn_rows failed ({rc})")
+    return out
+
+
+def flops(B, heads, T, H, W, d, win) -> float:
+    """Algorithmic FLOPs: sum over windows of 4 * n_m^2 * d, times B * heads."""
+    lib = _load()
+    w3 = _I3(*[int(a) for a in win])
+    return float(lib.oref_flops(int(B), int(heads), int(T), int(H), int(W), int(d), w3))

@@ -1,0 +1,487 @@
+/*
+ * oracle/ref_swattn.c -- fp64 CPU oracle for shifted local-window self-attention.
+ *
+ * TEST INFRASTRUCTURE, NOT PRODUCT CODE.  Only the test suite, the smoke check
+ * and the CPU-baseline leg of the benchmark load this library.  It shares no
+ * source, header, table or helper with the CUDA path; the two meet only in
+ * the seeded input generators, which hold none of the method's arithmetic.
+ *
+ * What it computes (paper: "Backend-Agnostic Sparse Attention for Fast
+ * High-Resolution Visual Generation", BASA):
+ *
+ *   §3.1 "Shifted Window Sparse Attention": at each sparse-attention layer the
+ *   token grid is cyclically shifted by -Delta, partitioned into
+ *   non-overlapping windows, standard scaled dot-product softmax attention is
+ *   applied inside each window with the unchanged Q/K/V, and the outputs are
+ *   merged and shifted back by +Delta to their original positions.
+ *
+ *   Appendix A.1 "Regular execution with standard attention backends": the
+ *   shift is a cyclic roll, the windows are formed by reshape/permute and
+ *   folded into the batch dimension, each folded window is one dense
+ *   attention problem.
+ *
+ * The four stages are carried out one after the other, each materialising its
+ * result, with no fusion:
+ *
+ *   1. roll      R[t',h',w'] = X[(t'+Dt) mod T, (h'+Dh) mod H, (w'+Dw) mod W]
+ *                (a roll by -Delta, the numpy/torch "roll(x, -Delta)" rule)
+ *   2. partition windows are the boxes [m_a*w_a, min((m_a+1)*w_a, n_a)) of the
+ *                rolled grid along each axis a, numbered in raster order over
+ *                (m_t, m_h, m_w); slots inside a window are numbered in raster
+ *                order over (s_t, s_h, s_w).
+ *   3. attend    per (batch item, window, head): S = scale * Q_w K_w^T,
+ *                P = softmax(S) row-wise (max-subtracted), O_w = P V_w, fp64.
+ *   4. merge     window outputs are written back to their rolled positions,
+ *      + unroll  and the grid is rolled by +Delta: Y[p] = R_O[(p - Delta) mod n].
+ *
+ * Readings where the pages are silent (each also listed in the design notes):
+ *   - the same cyclic rule applies on the temporal axis when w_t < T;
+ *   - a grid that the window does not divide gets a truncated last window
+ *     along that axis (no padded tokens take part in any softmax);
+ *   - every head and every batch item uses the same partition;
+ *   - the inputs are bf16 bit patterns, widened exactly to fp64.
+ *
+ * Data layout: Q, K, V are bf16 [B, T*H*W, heads, d] (raster token order t,h,w),
+ * passed as uint16 bit patterns; the output is fp64 [B, T*H*W, heads, d].
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define OREF_OK 0
+#define OREF_ERR_ARG (-1)
+#define OREF_ERR_NOMEM (-2)
+
+/* ------------------------------------------------------------------ */
+/* scalar helpers                                                      */
+/* ------------------------------------------------------------------ */
+
+/* bf16 bit pattern -> fp64, exact (bf16 is the top half of an fp32). */
+static double bf16_to_f64(uint16_t bits)
+{
+    uint32_t u = (uint32_t)bits << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* mathematical modulus: result in [0, n) for any integer a and n > 0 */
+static long pmod(long a, long n)
+{
+    long r = a % n;
+    return r < 0 ? r + n : r;
+}
+
+/* ------------------------------------------------------------------ */
+/* geometry                                                            */
+/* ------------------------------------------------------------------ */
+
+typedef struct {
+    int n[3];      /* grid extent (T, H, W)                    */
+    int w[3];      /* window extent (w_t, w_h, w_w)            */
+    int delta[3];  /* shift Delta reduced into [0, n_a)        */
+    int nwin[3];   /* windows per axis, ceil(n_a / w_a)        */
+    long N;        /* tokens in the grid                       */
+    long n_windows;/* windows in the grid                      */
+    int nw_max;    /* tokens in a full window                  */
+} geom_t;
+
+static int geom_init(geom_t *g, int T, int H, int W, const int win[3], const int shift[3])
+{
+    int a;
+    if (T < 1 || H < 1 || W < 1 || !win || !shift) return OREF_ERR_ARG;
+    g->n[0] = T; g->n[1] = H; g->n[2] = W;
+    g->N = (long)T * H * W;
+    g->n_windows = 1;
+    g->nw_max = 1;
+    for (a = 0; a < 3; ++a) {
+        if (win[a] < 1 || win[a] > g->n[a]) return OREF_ERR_ARG;
+        g->w[a] = win[a];
+        g->delta[a] = (int)pmod(shift[a], g->n[a]);
+        g->nwin[a] = (g->n[a] + win[a] - 1) / win[a];
+        g->n_windows *= g->nwin[a];
+        g->nw_max *= win[a];
+    }
+    return OREF_OK;
+}
+
+/* extent of window index m_a along axis a: full, or truncated at the grid edge */
+static int window_extent(const geom_t *g, int a, int m_a)
+{
+    int start = m_a * g->w[a];
+    int left = g->n[a] - start;
+    return left < g->w[a] ? left : g->w[a];
+}
+
+/* ------------------------------------------------------------------ */
+/* stage 1 and stage 4b: cyclic roll of a (T, H, W, C) grid            */
+/* ------------------------------------------------------------------ */
+
+/*
+ * sign = -1: roll by -Delta, out[i] = in[(i + Delta) mod n]   (stage 1)
+ * sign = +1: roll by +Delta, out[i] = in[(i - Delta) mod n]   (stage 4)
+ */
+static void roll_grid(const double *in, double *out, const geom_t *g, long C, int sign)
+{
+    int t, h, w;
+    for (t = 0; t < g->n[0]; ++t) {
+        long ts = pmod((long)t - (long)sign * g->delta[0], g->n[0]);
+        for (h = 0; h < g->n[1]; ++h) {
+            long hs = pmod((long)h - (long)sign * g->delta[1], g->n[1]);
+            for (w = 0; w < g->n[2]; ++w) {
+                long wsrc = pmod((long)w - (long)sign * g->delta[2], g->n[2]);
+                long dst = ((long)t * g->n[1] + h) * g->n[2] + w;
+                long src = (ts * g->n[1] + hs) * g->n[2] + wsrc;
+                memcpy(out + dst * C, in + src * C, (size_t)C * sizeof(double));
+            }
+        }
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* stage 2 and stage 4a: partition into windows, and its inverse       */
+/* ------------------------------------------------------------------ */
+
+/*
+ * Window m (raster over m_t, m_h, m_w) of the rolled grid is copied into
+ * wbuf[m][slot][C] with slots in raster order; count[m] receives its size.
+ * to_windows = 0 performs the inverse copy (merge).
+ */
+static void partition_grid(double *grid, double *wbuf, int *count, const geom_t *g, long C,
+                           int to_windows)
+{
+    long m = 0;
+    int mt, mh, mw, st, sh, sw;
+    for (mt = 0; mt < g->nwin[0]; ++mt)
+        for (mh = 0; mh < g->nwin[1]; ++mh)
+            for (mw = 0; mw < g->nwin[2]; ++mw, ++m) {
+                int et = window_extent(g, 0, mt);
+                int eh = window_extent(g, 1, mh);
+                int ew = window_extent(g, 2, mw);
+                long slot = 0;
+                for (st = 0; st < et; ++st)
+                    for (sh = 0; sh < eh; ++sh)
+                        for (sw = 0; sw < ew; ++sw, ++slot) {
+                            long t = (long)mt * g->w[0] + st;
+                            long h = (long)mh * g->w[1] + sh;
+                            long w = (long)mw * g->w[2] + sw;
+                            double *gp = grid + ((t * g->n[1] + h) * g->n[2] + w) * C;
+                            double *wp = wbuf + (m * g->nw_max + slot) * C;
+                            if (to_windows)
+                                memcpy(wp, gp, (size_t)C * sizeof(double));
+                            else
+                                memcpy(gp, wp, (size_t)C * sizeof(double));
+                        }
+                if (count) count[m] = (int)slot;
+            }
+}
+
+/* ------------------------------------------------------------------ */
+/* stage 3: dense softmax attention inside one window                  */
+/* ------------------------------------------------------------------ */
+
+/*
+ * q, k, v, o: [n][d] row-major fp64.  S = scale * q k^T; each row of S goes
+ * through a max-subtracted softmax; o = P v.  work holds n doubles.
+ */
+static void window_attention(const double *q, const double *k, const double *v, double *o,
+                             int n, int d, double scale, double *work)
+{
+    int i, j, c;
+    for (i = 0; i < n; ++i) {
+        double mx = -INFINITY, sum = 0.0;
+        for (j = 0; j < n; ++j) {
+            double s = 0.0;
+            for (c = 0; c < d; ++c) s += q[(long)i * d + c] * k[(long)j * d + c];
+            work[j] = scale * s;
+            if (work[j] > mx) mx = work[j];
+        }
+        for (j = 0; j < n; ++j) {
+            work[j] = exp(work[j] - mx);
+            sum += work[j];
+        }
+        for (c = 0; c < d; ++c) o[(long)i * d + c] = 0.0;
+        for (j = 0; j < n; ++j) {
+            double p = work[j] / sum;
+            for (c = 0; c < d; ++c) o[(long)i * d + c] += p * v[(long)j * d + c];
+        }
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* index map: which original token sits in (window, slot)              */
+/* ------------------------------------------------------------------ */
+
+/*
+ * token_of_slot: [n_windows][nw_max] int32, -1 where a truncated window has
+ * no token in that slot.  count_of_window: [n_windows] int32 (may be NULL).
+ * Computed by pushing the raster ids of the tokens through stages 1 and 2.
+ */
+int oref_index_map(int T, int H, int W, const int win[3], const int shift[3],
+                   int32_t *token_of_slot, int32_t *count_of_window)
+{
+    geom_t g;
+    double *ids, *rolled, *wbuf;
+    int *count;
+    long i;
+    int rc = geom_init(&g, T, H, W, win, shift);
+    if (rc) return rc;
+    if (!token_of_slot) return OREF_ERR_ARG;
+    ids = (double *)malloc(sizeof(double) * (size_t)g.N);
+    rolled = (double *)malloc(sizeof(double) * (size_t)g.N);
+    wbuf = (double *)malloc(sizeof(double) * (size_t)(g.n_windows * g.nw_max));
+    count = (int *)malloc(sizeof(int) * (size_t)g.n_windows);
+    if (!ids || !rolled || !wbuf || !count) {
+        free(ids); free(rolled); free(wbuf); free(count);
+        return OREF_ERR_NOMEM;
+    }
+    for (i = 0; i < g.N; ++i) ids[i] = (double)i;
+    for (i = 0; i < g.n_windows * g.nw_max; ++i) wbuf[i] = -1.0;
+    roll_grid(ids, rolled, &g, 1, -1);
+    partition_grid(rolled, wbuf, count, &g, 1, 1);
+    for (i = 0; i < g.n_windows * g.nw_max; ++i) token_of_slot[i] = (int32_t)wbuf[i];
+    if (count_of_window)
+        for (i = 0; i < g.n_windows; ++i) count_of_window[i] = count[i];
+    free(ids); free(rolled); free(wbuf); free(count);
+    return OREF_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* the full forward                                                    */
+/* ------------------------------------------------------------------ */
+
+typedef struct {
+    const geom_t *g;
+    const double *qw, *kw, *vw; /* [n_windows][nw_max][d] for one (b, head) */
+    double *ow;
+    const int *count;
+    int d;
+    double scale;
+    long next;                  /* shared window counter */
+    int failed;
+} attn_job_t;
+
+static void *attn_worker(void *arg)
+{
+    attn_job_t *job = (attn_job_t *)arg;
+    double *work = (double *)malloc(sizeof(double) * (size_t)job->g->nw_max);
+    if (!work) {
+        __atomic_store_n(&job->failed, 1, __ATOMIC_SEQ_CST);
+        return NULL;
+    }
+    for (;;) {
+        long m = __atomic_fetch_add(&job->next, 1, __ATOMIC_SEQ_CST);
+        long off;
+        if (m >= job->g->n_windows) break;
+        off = m * job->g->nw_max * job->d;
+        window_attention(job->qw + off, job->kw + off, job->vw + off, job->ow + off,
+                         job->count[m], job->d, job->scale, work);
+    }
+    free(work);
+    return NULL;
+}
+
+/*
+ * out[b, token, head, :] for head in [head_begin, head_end); other heads of
+ * out are left untouched.  nthreads <= 0 means one thread.
+ */
+int oref_swattn_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, double *out,
+                    int B, int heads, int T, int H, int W, int d,
+                    const int win[3], const int shift[3], double scale,
+                    int head_begin, int head_end, int nthreads)
+{
+    geom_t g;
+    long N, wsz, tok, c;
+    int b, hd, i, rc;
+    double *xq, *xk, *xv, *rq, *rk, *rv, *wq, *wk, *wv, *wo, *ro, *y;
+    int *count;
+    rc = geom_init(&g, T, H, W, win, shift);
+    if (rc) return rc;
+    if (!q || !k || !v || !out || B < 1 || heads < 1 || d < 1) return OREF_ERR_ARG;
+    if (head_begin < 0 || head_end > heads || head_begin >= head_end) return OREF_ERR_ARG;
+    if (nthreads < 1) nthreads = 1;
+    N = g.N;
+    wsz = g.n_windows * g.nw_max * d;
+    xq = (double *)malloc(sizeof(double) * (size_t)(N * d));
+    xk = (double *)malloc(sizeof(double) * (size_t)(N * d));
+    xv = (double *)malloc(sizeof(double) * (size_t)(N * d));
+    rq = (double *)malloc(sizeof(double) * (size_t)(N * d));
+    rk = (double *)malloc(sizeof(double) * (size_t)(N * d));
+    rv = (double *)malloc(sizeof(double) * (size_t)(N * d));
+    ro = (double *)malloc(sizeof(double) * (size_t)(N * d));
+    y = (double *)malloc(sizeof(double) * (size_t)(N * d));
+    wq = (double *)calloc((size_t)wsz, sizeof(double));
+    wk = (double *)calloc((size_t)wsz, sizeof(double));
+    wv = (double *)calloc((size_t)wsz, sizeof(double));
+    wo = (double *)calloc((size_t)wsz, sizeof(double));
+    count = (int *)malloc(sizeof(int) * (size_t)g.n_windows);
+    rc = OREF_OK;
+    if (!xq || !xk || !xv || !rq || !rk || !rv || !ro || !y || !wq || !wk || !wv || !wo || !count) {
+        rc = OREF_ERR_NOMEM;
+        goto done;
+    }
+    for (b = 0; b < B; ++b) {
+        for (hd = head_begin; hd < head_end; ++hd) {
+            pthread_t *tids;
+            attn_job_t job;
+            /* this head's grid, widened to fp64 */
+            for (tok = 0; tok < N; ++tok) {
+                long src = (((long)b * N + tok) * heads + hd) * d;
+                for (c = 0; c < d; ++c) {
+                    xq[tok * d + c] = bf16_to_f64(q[src + c]);
+                    xk[tok * d + c] = bf16_to_f64(k[src + c]);
+                    xv[tok * d + c] = bf16_to_f64(v[src + c]);
+                }
+            }
+            /* stage 1: roll by -Delta */
+            roll_grid(xq, rq, &g, d, -1);
+            roll_grid(xk, rk, &g, d, -1);
+            roll_grid(xv, rv, &g, d, -1);
+            /* stage 2: partition */
+            partition_grid(rq, wq, count, &g, d, 1);
+            partition_grid(rk, wk, NULL, &g, d, 1);
+            partition_grid(rv, wv, NULL, &g, d, 1);
+            /* stage 3: attention in every window */
+            job.g = &g; job.qw = wq; job.kw = wk; job.vw = wv; job.ow = wo;
+            job.count = count; job.d = d; job.scale = scale; job.next = 0; job.failed = 0;
+            tids = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nthreads);
+            if (!tids) { rc = OREF_ERR_NOMEM; goto done; }
+            for (i = 0; i < nthreads; ++i)
+                if (pthread_create(&tids[i], NULL, attn_worker, &job) != 0) break;
+            {
+                int started = i, j;
+                if (started == 0) attn_worker(&job);
+                for (j = 0; j < started; ++j) pthread_join(tids[j], NULL);
+            }
+            free(tids);
+            if (job.failed) { rc = OREF_ERR_NOMEM; goto done; }
+            /* stage 4: merge, then roll back by +Delta */
+            partition_grid(ro, wo, NULL, &g, d, 0);
+            roll_grid(ro, y, &g, d, +1);
+            for (tok = 0; tok < N; ++tok) {
+                long dst = (((long)b * N + tok) * heads + hd) * d;
+                memcpy(out + dst, y + tok * d, sizeof(double) * (size_t)d);
+            }
+        }
+    }
+done:
+    free(xq); free(xk); free(xv); free(rq); free(rk); free(rv); free(ro); free(y);
+    free(wq); free(wk); free(wv); free(wo); free(count);
+    return rc;
+}
+
+/* ------------------------------------------------------------------ */
+/* single output rows, for sampling large grids                        */
+/* ------------------------------------------------------------------ */
+
+/*
+ * For each requested (b, token, head) triple, the same four stages restricted
+ * to one query: the query's rolled position (stage 1), the window that holds
+ * it and that window's tokens in slot order (stage 2), one softmax row over
+ * the window (stage 3), and the result returned for the token it came from
+ * (stage 4).  out_rows: [nrows][d].  Arithmetic order per row equals
+ * oref_swattn_fwd's, so the two agree bit for bit.
+ */
+int oref_swattn_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                     int B, int heads, int T, int H, int W, int d,
+                     const int win[3], const int shift[3], double scale,
+                     const int64_t *triples, long nrows, double *out_rows)
+{
+    geom_t g;
+    long r;
+    int rc = geom_init(&g, T, H, W, win, shift);
+    double *kw, *vw, *qrow, *work;
+    if (rc) return rc;
+    if (!q || !k || !v || !triples || !out_rows || B < 1 || heads < 1 || d < 1) return OREF_ERR_ARG;
+    kw = (double *)malloc(sizeof(double) * (size_t)g.nw_max * d);
+    vw = (double *)malloc(sizeof(double) * (size_t)g.nw_max * d);
+    qrow = (double *)malloc(sizeof(double) * (size_t)d);
+    work = (double *)malloc(sizeof(double) * (size_t)g.nw_max);
+    if (!kw || !vw || !qrow || !work) {
+        free(kw); free(vw); free(qrow); free(work);
+        return OREF_ERR_NOMEM;
+    }
+    for (r = 0; r < nrows; ++r) {
+        long b = triples[3 * r], tok = triples[3 * r + 1], hd = triples[3 * r + 2];
+        long p[3], rp[3], m[3], e[3], c, j, n;
+        double mx = -INFINITY, sum = 0.0;
+        if (b < 0 || b >= B || tok < 0 || tok >= g.N || hd < 0 || hd >= heads) {
+            rc = OREF_ERR_ARG;
+            break;
+        }
+        p[0] = tok / ((long)g.n[1] * g.n[2]);
+        p[1] = (tok / g.n[2]) % g.n[1];
+        p[2] = tok % g.n[2];
+        /* stage 1: after the roll by -Delta the token sits at (p - Delta) mod n */
+        for (c = 0; c < 3; ++c) {
+            rp[c] = pmod(p[c] - g.delta[c], g.n[c]);
+            m[c] = rp[c] / g.w[c];                   /* stage 2: its window */
+            e[c] = window_extent(&g, (int)c, (int)m[c]);
+        }
+        /* stage 2: the window's tokens in slot order (rolled coordinate + Delta) */
+        n = 0;
+        {
+            long st, sh, sw;
+            for (st = 0; st < e[0]; ++st)
+                for (sh = 0; sh < e[1]; ++sh)
+                    for (sw = 0; sw < e[2]; ++sw, ++n) {
+                        long ot = pmod(m[0] * g.w[0] + st + g.delta[0], g.n[0]);
+                        long oh = pmod(m[1] * g.w[1] + sh + g.delta[1], g.n[1]);
+                        long ow = pmod(m[2] * g.w[2] + sw + g.delta[2], g.n[2]);
+                        long otok = (ot * g.n[1] + oh) * g.n[2] + ow;
+                        long src = ((b * g.N + otok) * heads + hd) * d;
+                        for (c = 0; c < d; ++c) {
+                            kw[n * d + c] = bf16_to_f64(k[src + c]);
+                            vw[n * d + c] = bf16_to_f64(v[src + c]);
+                        }
+                    }
+        }
+        {
+            long src = ((b * g.N + tok) * heads + hd) * d;
+            for (c = 0; c < d; ++c) qrow[c] = bf16_to_f64(q[src + c]);
+        }
+        /* stage 3: one softmax row, same operation order as window_attention */
+        for (j = 0; j < n; ++j) {
+            double s = 0.0;
+            for (c = 0; c < d; ++c) s += qrow[c] * kw[j * d + c];
+            work[j] = scale * s;
+            if (work[j] > mx) mx = work[j];
+        }
+        for (j = 0; j < n; ++j) {
+            work[j] = exp(work[j] - mx);
+            sum += work[j];
+        }
+        for (c = 0; c < d; ++c) out_rows[r * d + c] = 0.0;
+        for (j = 0; j < n; ++j) {
+            double pj = work[j] / sum;
+            for (c = 0; c < d; ++c) out_rows[r * d + c] += pj * vw[j * d + c];
+        }
+        /* stage 4: the row belongs to the token it was gathered from */
+    }
+    free(kw); free(vw); free(qrow); free(work);
+    return rc;
+}
+
+/*
+ * Algorithmic FLOPs of the windowed forward: every window contributes
+ * 4 * n_m^2 * d per head and batch item (2 n_m^2 d for Q K^T, 2 n_m^2 d for P V),
+ * following the O(N n_w d) cost in §3.1 "Attention complexity".
+ */
+double oref_flops(int B, int heads, int T, int H, int W, int d, const int win[3])
+{
+    geom_t g;
+    int zero[3] = {0, 0, 0};
+    int mt, mh, mw;
+    double total = 0.0;
+    if (geom_init(&g, T, H, W, win, zero)) return -1.0;
+    for (mt = 0; mt < g.nwin[0]; ++mt)
+        for (mh = 0; mh < g.nwin[1]; ++mh)
+            for (mw = 0; mw < g.nwin[2]; ++mw) {
+                double n = (double)window_extent(&g, 0, mt) * window_extent(&g, 1, mh) *
+                           window_extent(&g, 2, mw);
+                total += 4.0 * n * n * d;
+            }
+    return total * B * heads;
+}

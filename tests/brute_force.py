@@ -1,0 +1,58 @@
+"""Independent numpy formulations used to pin the oracle (tiny sizes only).
+
+Shifted-window attention is restated here in a second, differently built form:
+full attention over the ORIGINAL token order with a block-diagonal mask, where
+two tokens may attend to each other iff they fall into the same window after
+the grid is rolled by -Delta ("Backend-Agnostic Sparse Attention for Fast
+High-Resolution Visual Generation", §3.1 "Shifted Window Sparse Attention").
+Window membership comes from ``numpy.roll`` of a grid of token ids, not from the
+oracle's index arithmetic.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    """uint16 bf16 bit patterns -> fp64 (exact)."""
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def window_id_of_token(T, H, W, win, shift) -> np.ndarray:
+    """[N] window id of every original token.
+
+    numpy.roll(ids, -Delta) puts original token (i + Delta) mod n at position i;
+    position i of the rolled grid lies in window (i_t // w_t, i_h // w_h, i_w // w_w).
+    """
+    ids = np.arange(T * H * W).reshape(T, H, W)
+    rolled = np.roll(ids, shift=(-shift[0], -shift[1], -shift[2]), axis=(0, 1, 2))
+    nwin = [-(-n // w) for n, w in zip((T, H, W), win)]
+    ct, ch, cw = np.meshgrid(np.arange(T) // win[0], np.arange(H) // win[1],
+                             np.arange(W) // win[2], indexing="ij")
+    wid_at_pos = (ct * nwin[1] + ch) * nwin[2] + cw
+    out = np.empty(T * H * W, dtype=np.int64)
+    out[rolled.reshape(-1)] = wid_at_pos.reshape(-1)
+    return out
+
+
+def full_attention(q, k, v, scale, mask=None):
+    """Plain softmax attention per (b, head): q, k, v fp64 [B, N, heads, d]."""
+    B, N, heads, d = q.shape
+    out = np.empty_like(q)
+    for b in range(B):
+        for h in range(heads):
+            s = scale * (q[b, :, h, :] @ k[b, :, h, :].T)
+            if mask is not None:
+                s = np.where(mask, s, -np.inf)
+            s = s - s.max(axis=1, keepdims=True)
+            p = np.exp(s)
+            p /= p.sum(axis=1, keepdims=True)
+            out[b, :, h, :] = p @ v[b, :, h, :]
+    return out
+
+
+def masked_window_attention(q, k, v, T, H, W, win, shift, scale):
+    """Shifted-window attention as block-diagonally masked full attention."""
+    wid = window_id_of_token(T, H, W, win, shift)
+    mask = wid[:, None] == wid[None, :]
+    return full_attention(q, k, v, scale, mask)

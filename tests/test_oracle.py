@@ -1,0 +1,248 @@
+"""Pins of the fp64 oracle against facts that do not come from the oracle itself.
+
+Method: "Backend-Agnostic Sparse Attention for Fast High-Resolution Visual
+Generation" (BASA), §3.1 "Shifted Window Sparse Attention" (roll by -Delta,
+non-overlapping windows, softmax attention per window, roll back by +Delta),
+§3.1 "Attention complexity" and Table 3 (FLOP accounting).
+
+Each pin is chosen so that a plausible slip in the oracle fails at least one:
+  * the roll direction and window numbering -> hand-worked index maps;
+  * the softmax / scale / transposition     -> full-grid window equals plain
+    attention, two-token closed form;
+  * window membership and the un-roll        -> masked full attention built from
+    numpy.roll;
+  * truncated windows                         -> non-divisible grids in the
+    masked comparison and in the hand-worked 3D map;
+  * invariances the pages imply               -> shifts by whole windows or by
+    the grid size change nothing.
+"""
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from brute_force import (bf16_bits_to_f64, full_attention, masked_window_attention,
+                         window_id_of_token)
+from shifted_window_attention_swattn_b200.inputs import make_custom
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _qkv(B, heads, d, T, H, W, seed, dist="normal"):
+    q, k, v = make_custom(B, heads, d, T, H, W, seed, dist=dist)
+    bits = [oracle._bits(x) for x in (q, k, v)]
+    f64 = [bf16_bits_to_f64(b).reshape(B, T * H * W, heads, d) for b in bits]
+    return bits, f64
+
+
+def _read_index_cases():
+    cases, cur = [], None
+    with open(os.path.join(GOLDEN, "index_maps.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            if line.startswith("case"):
+                kv = dict(tok.split("=") for tok in line.split()[1:])
+                cur = {k: tuple(int(x) for x in v.split(",")) for k, v in kv.items()}
+                cur["rows"] = []
+            elif line == "end":
+                cases.append(cur)
+                cur = None
+            else:
+                cur["rows"].append([int(x) for x in line.split()])
+    return cases
+
+
+@pytest.mark.parametrize("case", _read_index_cases(), ids=lambda c: f"{c['grid']}-{c['shift']}")
+def test_index_map_matches_hand_worked_cases(case):
+    T, H, W = case["grid"]
+    tos, cnt = oracle.index_map(T, H, W, case["win"], case["shift"])
+    expect = np.array(case["rows"], dtype=np.int32)
+    np.testing.assert_array_equal(tos, expect)
+    np.testing.assert_array_equal(cnt, (expect >= 0).sum(axis=1))
+
+
+def test_roll_direction_is_observable():
+    # A shift that is not half the window must give a map that differs from
+    # the opposite shift, so a sign slip cannot hide behind symmetric cases.
+    a, _ = oracle.index_map(1, 4, 4, (1, 2, 2), (0, 1, 1))
+    b, _ = oracle.index_map(1, 4, 4, (1, 2, 2), (0, -1, -1))
+    assert not np.array_equal(a, b)
+
+
+@pytest.mark.parametrize("grid,win,shift", [
+    ((1, 6, 10), (1, 3, 4), (0, 2, 7)),
+    ((3, 5, 7), (2, 2, 3), (1, 4, 5)),
+    ((4, 4, 4), (4, 4, 4), (0, 0, 0)),
+    ((2, 3, 9), (1, 3, 9), (1, -1, -13)),
+    ((5, 1, 1), (2, 1, 1), (3, 0, 0)),
+])
+def test_index_map_is_bijection_consistent_with_numpy_roll(grid, win, shift):
+    T, H, W = grid
+    tos, cnt = oracle.index_map(T, H, W, win, shift)
+    valid = tos[tos >= 0]
+    assert sorted(valid.tolist()) == list(range(T * H * W))
+    wid = window_id_of_token(T, H, W, win, shift)
+    for m in range(tos.shape[0]):
+        members = tos[m, :cnt[m]]
+        assert np.all(wid[members] == m)
+        assert np.all(tos[m, cnt[m]:] == -1)
+
+
+@pytest.mark.parametrize("shift", [(0, 0, 0), (0, 3, 5), (1, -2, 9)])
+def test_window_equal_to_grid_is_full_attention(shift):
+    # Window = whole grid: the roll is a permutation and attention is
+    # permutation-equivariant, so the result is plain full attention.
+    B, heads, d, T, H, W = 2, 2, 16, 2, 5, 6
+    bits, (q, k, v) = _qkv(B, heads, d, T, H, W, seed=11)
+    scale = 1.0 / math.sqrt(d)
+    got = oracle.swattn_fwd(*bits, B, heads, T, H, W, d, (T, H, W), shift, scale)
+    ref = full_attention(q, k, v, scale)
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("grid,win,shift,d", [
+    ((1, 8, 8), (1, 4, 4), (0, 2, 2), 16),
+    ((1, 6, 10), (1, 3, 4), (0, 2, 7), 8),        # W not divisible by w_w
+    ((3, 5, 7), (2, 2, 3), (1, 4, 5), 8),         # 3D, nothing divisible
+    ((3, 4, 6), (3, 2, 3), (-1, 5, -4), 8),       # negative and oversized shifts
+    ((2, 3, 3), (1, 1, 1), (1, 1, 1), 4),         # one-token windows
+])
+def test_matches_masked_full_attention(grid, win, shift, d):
+    T, H, W = grid
+    B, heads = 2, 3
+    bits, (q, k, v) = _qkv(B, heads, d, T, H, W, seed=sum(grid) + d)
+    scale = 0.7 / math.sqrt(d)
+    got = oracle.swattn_fwd(*bits, B, heads, T, H, W, d, win, shift, scale)
+    ref = masked_window_attention(q, k, v, T, H, W, win, shift, scale)
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+
+
+def test_shift_by_whole_windows_is_bitwise_unshifted():
+    # Windows divide the grid: a shift by whole windows only relabels windows.
+    B, heads, d, T, H, W = 1, 2, 16, 2, 8, 12
+    win = (1, 4, 3)
+    bits, _ = _qkv(B, heads, d, T, H, W, seed=5)
+    base = oracle.swattn_fwd(*bits, B, heads, T, H, W, d, win, (0, 0, 0), 0.25)
+    for shift in [(1, 4, 3), (0, 8, 9), (1, -4, -6)]:
+        got = oracle.swattn_fwd(*bits, B, heads, T, H, W, d, win, shift, 0.25)
+        assert np.array_equal(got, base), shift
+
+
+def test_shift_by_grid_extent_is_identity():
+    B, heads, d, T, H, W = 1, 1, 8, 3, 5, 7
+    win = (2, 2, 3)
+    bits, _ = _qkv(B, heads, d, T, H, W, seed=6)
+    a = oracle.swattn_fwd(*bits, B, heads, T, H, W, d, win, (1, 2, 3), 0.3)
+    b = oracle.swattn_fwd(*bits, B, heads, T, H, W, d, win, (1 + T, 2 - 2 * H, 3 + 5 * W), 0.3)
+    assert np.array_equal(a, b)
+
+
+def test_scale_zero_gives_window_mean_of_v():
+    B, heads, d, T, H, W = 1, 2, 8, 2, 6, 5
+    win, shift = (2, 4, 2), (1, 3, 1)
+    bits, (_, _, v) = _qkv(B, heads, d, T, H, W, seed=7)
+    got = oracle.swattn_fwd(*bits, B, heads, T, H, W, d, win, shift, 0.0)
+    wid = window_id_of_token(T, H, W, win, shift)
+    ref = np.empty_like(v)
+    for m in np.unique(wid):
+        sel = wid == m
+        ref[:, sel] = v[:, sel].mean(axis=1, keepdims=True)
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-14)
+
+
+def test_constant_v_gives_constant_output():
+    B, heads, d, T, H, W = 1, 2, 8, 1, 6, 6
+    bits, _ = _qkv(B, heads, d, T, H, W, seed=8)
+    vconst = np.full_like(bits[2], 0x3FC0)   # bf16 1.5
+    got = oracle.swattn_fwd(bits[0], bits[1], vconst, B, heads, T, H, W, d, (1, 3, 2), (0, 1, 1), 1.0)
+    np.testing.assert_allclose(got, 1.5, rtol=0, atol=1e-14)
+
+
+def test_single_token_windows_return_v_exactly():
+    B, heads, d, T, H, W = 1, 2, 8, 2, 3, 4
+    bits, (_, _, v) = _qkv(B, heads, d, T, H, W, seed=9)
+    got = oracle.swattn_fwd(*bits, B, heads, T, H, W, d, (1, 1, 1), (1, 2, 3), 1.0)
+    assert np.array_equal(got, v)
+
+
+def test_two_token_window_closed_form():
+    # softmax over two keys: o = (e^{s1} v1 + e^{s2} v2) / (e^{s1} + e^{s2}).
+    B, heads, d, T, H, W = 1, 1, 4, 1, 1, 2
+    bits, (q, k, v) = _qkv(B, heads, d, T, H, W, seed=10)
+    scale = 0.5
+    got = oracle.swattn_fwd(*bits, B, heads, T, H, W, d, (1, 1, 2), (0, 0, 1), scale)
+    for i in range(2):
+        s = [scale * float(np.dot(q[0, i, 0], k[0, j, 0])) for j in range(2)]
+        e = [math.exp(x) for x in s]
+        o = (e[0] * v[0, 0, 0] + e[1] * v[0, 1, 0]) / (e[0] + e[1])
+        np.testing.assert_allclose(got[0, i, 0], o, rtol=1e-14, atol=1e-15)
+
+
+def test_rows_agree_bitwise_with_full_forward():
+    B, heads, d, T, H, W = 2, 3, 16, 3, 5, 7
+    win, shift = (2, 2, 3), (1, -2, 4)
+    bits, _ = _qkv(B, heads, d, T, H, W, seed=12)
+    full = oracle.swattn_fwd(*bits, B, heads, T, H, W, d, win, shift, 0.4)
+    rng = np.random.default_rng(0)
+    triples = np.stack([rng.integers(0, B, 40), rng.integers(0, T * H * W, 40),
+                        rng.integers(0, heads, 40)], axis=1)
+    rows = oracle.swattn_rows(*bits, B, heads, T, H, W, d, win, shift, 0.4, triples)
+    for r, (b, t, h) in enumerate(triples):
+        assert np.array_equal(rows[r], full[b, t, h])
+
+
+def test_head_range_leaves_other_heads_untouched():
+    B, heads, d, T, H, W = 1, 4, 8, 1, 4, 4
+    bits, _ = _qkv(B, heads, d, T, H, W, seed=13)
+    full = oracle.swattn_fwd(*bits, B, heads, T, H, W, d, (1, 2, 2), (0, 1, 1), 0.3)
+    part = oracle.swattn_fwd(*bits, B, heads, T, H, W, d, (1, 2, 2), (0, 1, 1), 0.3, head_range=(1, 3))
+    assert np.array_equal(part[:, :, 1:3], full[:, :, 1:3])
+    assert np.isnan(part[:, :, 0]).all() and np.isnan(part[:, :, 3]).all()
+
+
+def test_rejects_bad_geometry():
+    with pytest.raises(ValueError):
+        oracle.index_map(1, 4, 4, (1, 5, 2), (0, 0, 0))
+    with pytest.raises(ValueError):
+        oracle.index_map(1, 4, 4, (0, 2, 2), (0, 0, 0))
+
+
+def _read_flop_rows():
+    rows = []
+    with open(os.path.join(GOLDEN, "flop_counts.txt")) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                p = line.split()
+                rows.append((p[0], float(p[1]), [int(x) for x in p[2:]]))
+    return rows
+
+
+@pytest.mark.parametrize("row", _read_flop_rows(), ids=lambda r: r[0])
+def test_flop_metric_matches_printed_table(row):
+    name, printed_tflops, (T, H, W, heads, d, wt, wh, ww, terms) = row
+    local = oracle.flops(1, heads, T, H, W, d, (wt, wh, ww))
+    assert abs(terms * local / 1e12 - printed_tflops) / printed_tflops < 0.01
+
+
+def test_flops_closed_form_divisible_and_truncated():
+    # Divisible: 4 * N * n_w * d * heads * B.
+    assert oracle.flops(2, 3, 2, 8, 12, 16, (1, 4, 3)) == 4 * (2 * 8 * 12) * 12 * 16 * 3 * 2
+    # Truncated: sum over windows of 4 n_m^2 d; W = 5 cut into 2 + 2 + 1.
+    assert oracle.flops(1, 1, 1, 1, 5, 8, (1, 1, 2)) == 4 * 8 * (4 + 4 + 1)
+
+
+def test_masked_attention_helper_is_itself_sane():
+    # The brute force must reduce to plain attention when every token shares a
+    # window, and to identity when every window has one token.
+    B, heads, d, T, H, W = 1, 1, 4, 1, 2, 3
+    _, (q, k, v) = _qkv(B, heads, d, T, H, W, seed=14)
+    full = full_attention(q, k, v, 0.5)
+    np.testing.assert_allclose(
+        masked_window_attention(q, k, v, T, H, W, (T, H, W), (0, 0, 0), 0.5), full, atol=0)
+    np.testing.assert_allclose(
+        masked_window_attention(q, k, v, T, H, W, (1, 1, 1), (0, 1, 2), 0.5), v, atol=0)
