@@ -1,0 +1,115 @@
+/*
+ * basa_swattn.h -- C ABI of the B200 (sm_100a) shifted-window attention library
+ * (libbasa_swattn.so).
+ *
+ * Operation: the shifted local-window self-attention of "Backend-Agnostic
+ * Sparse Attention for Fast High-Resolution Visual Generation" (BASA),
+ * §3.1 "Shifted Window Sparse Attention": the visual token grid is cyclically
+ * shifted by -Delta, cut into non-overlapping windows, standard scaled
+ * dot-product softmax attention runs inside each window with the unchanged
+ * Q/K/V, and the outputs are merged and shifted back by +Delta.  Appendix A.1
+ * ("Regular execution with standard attention backends") describes the
+ * windows as dense attention problems folded into the batch; here the roll,
+ * the window gather, the attention and the inverse roll are one kernel.
+ *
+ * Conventions shared by every entry point
+ *   - Tensors Q, K, V and out are bf16, row-major [B, T*H*W, heads, d]; tokens
+ *     in raster order (t, h, w); d contiguous.  All four are DEVICE pointers,
+ *     16-byte aligned, owned by the caller; the library keeps no reference
+ *     after the call returns.
+ *   - win[3] and shift[3] are ordered (t, h, w).  1 <= win[a] <= extent[a].
+ *     A window that the grid does not divide is truncated at the grid edge
+ *     (the last window along that axis holds extent mod win tokens).
+ *   - shift[a] is any integer Delta_a; it is reduced modulo the extent.  The
+ *     grid is rolled by -Delta, so window m starts at original coordinate
+ *     (m_a * win[a] + Delta_a) mod extent[a] along each axis.
+ *   - Full attention is win = {T, H, W} with shift = {0, 0, 0}: one window.
+ *   - stream is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Launches are asynchronous; nothing is synchronised and nothing is
+ *     allocated per call.
+ *   - Errors are returned as BASA_* codes.  Argument errors are detected on
+ *     the host before anything is launched.  The library never prints, exits
+ *     or throws across this boundary.
+ */
+#ifndef BASA_SWATTN_H
+#define BASA_SWATTN_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define BASA_OK 0
+#define BASA_ERR_INVALID_ARG (-1)  /* null pointer, bad extent, window or size */
+#define BASA_ERR_UNSUPPORTED (-2)  /* head dim other than 64/128, too many rows, not sm_100 */
+#define BASA_ERR_ALIGNMENT (-3)    /* a tensor pointer is not 16-byte aligned */
+#define BASA_ERR_CUDA (-4)         /* a CUDA runtime or driver call failed */
+#define BASA_ERR_DEVICE (-5)       /* a bounded device-side wait expired in a launch */
+#define BASA_ERR_ALIAS (-6)        /* out overlaps q, k or v */
+
+/*
+ * Shifted-window attention forward (§3.1 "Shifted Window Sparse Attention").
+ *
+ *   q, k, v  in : device bf16 [B, T*H*W, heads, d]
+ *   out      out: device bf16 [B, T*H*W, heads, d]; must not overlap q, k or v
+ *   d        64 or 128
+ *   scale    softmax scale applied to Q K^T (1/sqrt(d) for standard attention)
+ *
+ * out[b, p, h, :] = sum_j softmax_j(scale * <q_p, k_j>) v_j over the tokens j
+ * that share the (shifted) window of token p.  Accumulation is fp32; P is
+ * rounded to bf16 before the P V product; the result is rounded to bf16.
+ * B * T*H*W * heads must be below 2^31.
+ */
+int basa_swattn_fwd(const void* q, const void* k, const void* v, void* out, int B, int heads,
+                    int T, int H, int W, int d, const int win[3], const int shift[3],
+                    float scale, void* stream);
+
+/*
+ * The index map of the shifted partition, computed on the device by the same
+ * device function the attention kernel uses for its gathers and scatters.
+ *
+ *   d_token_of_slot out: device int32 [n_windows, win[0]*win[1]*win[2]], the
+ *                        raster token index held by (window, slot); -1 in the
+ *                        slots a truncated window does not fill.
+ * Windows are numbered in raster order over (m_t, m_h, m_w) and slots in raster
+ * order over (s_t, s_h, s_w) of the rolled grid; n_windows is the product of
+ * ceil(extent[a] / win[a]).
+ */
+int basa_swattn_index_map(int T, int H, int W, const int win[3], const int shift[3],
+                          int32_t* d_token_of_slot, void* stream);
+
+/* The same index map computed on the host (same source function as the kernel's). */
+int basa_swattn_index_map_host(int T, int H, int W, const int win[3], const int shift[3],
+                               int32_t* token_of_slot);
+
+/*
+ * Algorithmic FLOPs of one forward (the O(N n_w d) cost of §3.1 "Attention
+ * complexity"): the sum over windows of 4 * n_m^2 * d, times B * heads, where
+ * n_m is the token count of window m.  Written to *flops.
+ */
+int basa_swattn_flops(int B, int heads, int T, int H, int W, int d, const int win[3],
+                      double* flops);
+
+/*
+ * Synchronises `stream`, then returns BASA_ERR_DEVICE if any launch since the
+ * previous call gave up on a bounded wait (BASA_OK otherwise), and clears the
+ * record.  Also returns BASA_ERR_CUDA if the synchronisation itself fails.
+ */
+int basa_swattn_last_device_error(void* stream);
+
+/*
+ * Upper bound, in nanoseconds, on every wait inside the kernels (default one
+ * second).  A launch whose wait runs out stops its work, drains what it has in
+ * flight, releases its tensor memory, and records BASA_ERR_DEVICE.
+ */
+int basa_swattn_set_wait_timeout_ns(unsigned long long ns);
+
+/* Static, human-readable text for a BASA_* code. */
+const char* basa_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BASA_SWATTN_H */

@@ -1,0 +1,215 @@
+"""B200 (sm_100a) shifted local-window self-attention.
+
+A thin ctypes binding over ``libbasa_swattn.so`` (C ABI in ``include/basa_swattn.h``).
+Python only checks and marshals arguments; the roll, window gather, attention
+and inverse roll all run in the CUDA kernel.  PyTorch supplies device memory
+and streams.  There is no CPU fallback: if the library is missing or fails to
+load, every call raises.
+
+Method: "Backend-Agnostic Sparse Attention for Fast High-Resolution Visual
+Generation" (BASA), §3.1 "Shifted Window Sparse Attention".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+__all__ = [
+    "swattn_fwd", "swattn_fwd_from_host", "index_map", "index_map_host", "flops",
+    "last_device_error", "set_wait_timeout_ns", "strerror", "library_path", "SwattnError",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_NAME = "libbasa_swattn.so"
+_lib = None
+_lock = threading.Lock()
+_I3 = ctypes.c_int * 3
+
+BASA_OK = 0
+BASA_ERR_INVALID_ARG = -1
+BASA_ERR_UNSUPPORTED = -2
+BASA_ERR_ALIGNMENT = -3
+BASA_ERR_CUDA = -4
+BASA_ERR_DEVICE = -5
+BASA_ERR_ALIAS = -6
+
+
+class SwattnError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {strerror(code)} ({code})")
+
+
+def library_path() -> str:
+    return os.path.join(_HERE, _LIB_NAME)
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        path = library_path()
+        if not os.path.exists(path):
+            raise RuntimeError(
+                f"{_LIB_NAME} is not built ({path}); run "
+                "`python -m shifted_window_attention_swattn_b200.build`")
+        lib = ctypes.CDLL(path)
+        vp, ci = ctypes.c_void_p, ctypes.c_int
+        lib.basa_swattn_fwd.argtypes = [vp, vp, vp, vp] + [ci] * 6 + [_I3, _I3, ctypes.c_float, vp]
+        lib.basa_swattn_fwd.restype = ci
+        lib.basa_swattn_index_map.argtypes = [ci, ci, ci, _I3, _I3, vp, vp]
+        lib.basa_swattn_index_map.restype = ci
+        lib.basa_swattn_index_map_host.argtypes = [ci, ci, ci, _I3, _I3, vp]
+        lib.basa_swattn_index_map_host.restype = ci
+        lib.basa_swattn_flops.argtypes = [ci] * 6 + [_I3, ctypes.POINTER(ctypes.c_double)]
+        lib.basa_swattn_flops.restype = ci
+        lib.basa_swattn_last_device_error.argtypes = [vp]
+        lib.basa_swattn_last_device_error.restype = ci
+        lib.basa_swattn_set_wait_timeout_ns.argtypes = [ctypes.c_ulonglong]
+        lib.basa_swattn_set_wait_timeout_ns.restype = ci
+        lib.basa_strerror.argtypes = [ci]
+        lib.basa_strerror.restype = ctypes.c_char_p
+        _lib = lib
+        return lib
+
+
+def strerror(code: int) -> str:
+    return _load().basa_strerror(int(code)).decode()
+
+
+def _triple(x, what):
+    t = tuple(int(a) for a in x)
+    if len(t) != 3:
+        raise ValueError(f"{what} must be a (t, h, w) triple")
+    return t
+
+
+def _stream_handle(stream, device):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def swattn_fwd(q, k, v, grid, win, shift, scale=None, out=None, stream=None):
+    """Shifted-window attention forward on device tensors.
+
+    q, k, v: bf16 CUDA tensors [B, T*H*W, heads, d] (contiguous), grid = (T, H, W),
+    win and shift (t, h, w) triples.  Returns ``out`` (allocated if not given).
+    Asynchronous on ``stream`` (default: the current stream of q's device).
+    """
+    import torch
+    lib = _load()
+    T, H, W = _triple(grid, "grid")
+    w3, s3 = _triple(win, "win"), _triple(shift, "shift")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or not t.is_cuda:
+            raise TypeError(f"{name} must be a bf16 CUDA tensor")
+        if not t.is_contiguous() or t.dim() != 4:
+            raise ValueError(f"{name} must be contiguous [B, T*H*W, heads, d]")
+    if q.shape != k.shape or q.shape != v.shape:
+        raise ValueError("q, k, v must have the same shape")
+    B, N, heads, d = q.shape
+    if N != T * H * W:
+        raise ValueError(f"token count {N} != T*H*W = {T * H * W}")
+    if out is None:
+        out = torch.empty_like(q)
+    elif out.shape != q.shape or out.dtype != torch.bfloat16 or not out.is_contiguous():
+        raise ValueError("out must be a contiguous bf16 tensor shaped like q")
+    if scale is None:
+        scale = d ** -0.5
+    rc = lib.basa_swattn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, heads,
+                             T, H, W, d, _I3(*w3), _I3(*s3), float(scale),
+                             _stream_handle(stream, q.device))
+    if rc != BASA_OK:
+        raise SwattnError(rc, "basa_swattn_fwd")
+    return out
+
+
+def swattn_fwd_from_host(q_host, k_host, v_host, grid, win, shift, scale=None, out_host=None,
+                         device="cuda", stream=None, dev_bufs=None):
+    """The same forward for inputs in host memory: H2D copy, kernel, D2H copy.
+
+    q_host, k_host, v_host: bf16 CPU tensors (pinned for asynchronous copies).
+    ``dev_bufs`` = (q, k, v, out) device tensors may be passed to reuse memory.
+    Returns the host output tensor; the call synchronises the stream.
+    """
+    import torch
+    if dev_bufs is None:
+        dev_bufs = tuple(torch.empty(q_host.shape, dtype=torch.bfloat16, device=device)
+                         for _ in range(4))
+    qd, kd, vd, od = dev_bufs
+    if stream is None:
+        stream = torch.cuda.current_stream(qd.device)
+    with torch.cuda.stream(stream):
+        qd.copy_(q_host, non_blocking=True)
+        kd.copy_(k_host, non_blocking=True)
+        vd.copy_(v_host, non_blocking=True)
+        swattn_fwd(qd, kd, vd, grid, win, shift, scale, out=od, stream=stream)
+        if out_host is None:
+            out_host = torch.empty(q_host.shape, dtype=torch.bfloat16, pin_memory=True)
+        out_host.copy_(od, non_blocking=True)
+    stream.synchronize()
+    return out_host
+
+
+def index_map(grid, win, shift, device="cuda", stream=None):
+    """Device-computed token_of_slot [n_windows, w_t*w_h*w_w] int32 (-1 padded)."""
+    import torch
+    lib = _load()
+    T, H, W = _triple(grid, "grid")
+    w3, s3 = _triple(win, "win"), _triple(shift, "shift")
+    if min(w3) < 1 or min(T, H, W) < 1:
+        raise ValueError("extents must be >= 1")
+    nwin = 1
+    for n, w in zip((T, H, W), w3):
+        nwin *= -(-n // w)
+    out = torch.empty((nwin, w3[0] * w3[1] * w3[2]), dtype=torch.int32, device=device)
+    rc = lib.basa_swattn_index_map(T, H, W, _I3(*w3), _I3(*s3), out.data_ptr(),
+                                   _stream_handle(stream, out.device))
+    if rc != BASA_OK:
+        raise SwattnError(rc, "basa_swattn_index_map")
+    return out
+
+
+def index_map_host(grid, win, shift):
+    """Host-computed token_of_slot (same source function as the kernel's)."""
+    import numpy as np
+    lib = _load()
+    T, H, W = _triple(grid, "grid")
+    w3, s3 = _triple(win, "win"), _triple(shift, "shift")
+    if min(w3) < 1 or min(T, H, W) < 1:
+        raise SwattnError(BASA_ERR_INVALID_ARG, "basa_swattn_index_map_host")
+    nwin = 1
+    for n, w in zip((T, H, W), w3):
+        nwin *= -(-n // w)
+    out = np.empty((nwin, w3[0] * w3[1] * w3[2]), dtype=np.int32)
+    rc = lib.basa_swattn_index_map_host(T, H, W, _I3(*w3), _I3(*s3), out.ctypes.data)
+    if rc != BASA_OK:
+        raise SwattnError(rc, "basa_swattn_index_map_host")
+    return out
+
+
+def flops(B, heads, grid, d, win) -> float:
+    """Algorithmic FLOPs of one forward: sum over windows of 4 n_m^2 d, times B*heads."""
+    lib = _load()
+    T, H, W = _triple(grid, "grid")
+    res = ctypes.c_double(0.0)
+    rc = lib.basa_swattn_flops(int(B), int(heads), T, H, W, int(d), _I3(*_triple(win, "win")),
+                               ctypes.byref(res))
+    if rc != BASA_OK:
+        raise SwattnError(rc, "basa_swattn_flops")
+    return res.value
+
+
+def last_device_error(stream=None) -> int:
+    """Synchronise and return (and clear) the device-side wait-timeout record."""
+    import torch
+    return _load().basa_swattn_last_device_error(
+        _stream_handle(stream, torch.device("cuda", torch.cuda.current_device())))
+
+
+def set_wait_timeout_ns(ns: int) -> None:
+    _load().basa_swattn_set_wait_timeout_ns(int(ns))

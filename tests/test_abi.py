@@ -1,0 +1,130 @@
+"""CPU-side checks of the C ABI library: it loads, exports every declared
+symbol, and its host logic (index map, FLOP count, argument validation) agrees
+with the oracle.  No kernel is launched here.
+"""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+import shifted_window_attention_swattn_b200 as sw
+from shifted_window_attention_swattn_b200 import build as sw_build
+from shifted_window_attention_swattn_b200.inputs import WORKLOADS
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+I3 = ctypes.c_int * 3
+
+
+@pytest.fixture(scope="module")
+def lib():
+    sw_build.build()
+    return sw._load()
+
+
+def _declared_functions():
+    names = []
+    inc = os.path.join(ROOT, "include")
+    for fn in sorted(os.listdir(inc)):
+        if fn.endswith(".h"):
+            text = open(os.path.join(inc, fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"\b(basa_\w+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_header_declares_the_entry_points():
+    names = _declared_functions()
+    for must in ("basa_swattn_fwd", "basa_swattn_index_map", "basa_swattn_flops",
+                 "basa_swattn_last_device_error", "basa_strerror"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_library_is_built_for_sm100a():
+    cmd = " ".join(sw_build.command("x.so"))
+    assert "arch=compute_100a,code=sm_100a" in cmd
+
+
+@pytest.mark.parametrize("wl", WORKLOADS, ids=lambda w: w.name)
+def test_host_index_map_equals_oracle_on_workloads(lib, wl):
+    for shift in wl.shifts:
+        got = sw.index_map_host(wl.grid, wl.win, shift)
+        ref, _ = oracle.index_map(*wl.grid, wl.win, shift)
+        assert np.array_equal(got, ref), shift
+
+
+@pytest.mark.parametrize("grid,win,shift", [
+    ((1, 4, 4), (1, 2, 2), (0, 1, 1)),
+    ((3, 1, 5), (2, 1, 2), (1, 0, 2)),
+    ((5, 9, 11), (2, 4, 5), (1, 7, -3)),
+    ((1, 20, 28), (1, 7, 9), (0, 3, 5)),
+    ((2, 16, 20), (2, 16, 10), (1, 8, 5)),
+    ((4, 6, 6), (4, 6, 6), (3, -2, 100)),
+    ((7, 3, 2), (1, 1, 1), (6, 2, 1)),
+])
+def test_host_index_map_equals_oracle(lib, grid, win, shift):
+    got = sw.index_map_host(grid, win, shift)
+    ref, _ = oracle.index_map(*grid, win, shift)
+    assert np.array_equal(got, ref)
+
+
+@pytest.mark.parametrize("wl", WORKLOADS, ids=lambda w: w.name)
+def test_flops_equal_oracle(lib, wl):
+    assert sw.flops(wl.B, wl.heads, wl.grid, wl.d, wl.win) == oracle.flops(
+        wl.B, wl.heads, *wl.grid, wl.d, wl.win)
+    full = sw.flops(wl.B, wl.heads, wl.grid, wl.d, wl.grid)
+    assert full == 4.0 * wl.N * wl.N * wl.d * wl.heads * wl.B
+
+
+def test_flops_truncated_windows(lib):
+    for grid, win in [((3, 5, 7), (2, 2, 3)), ((1, 20, 28), (1, 7, 9))]:
+        assert sw.flops(2, 3, grid, 64, win) == oracle.flops(2, 3, *grid, 64, win)
+
+
+def _fwd(lib, q=16, k=32, v=48, out=4096, B=1, heads=1, grid=(1, 4, 4), d=64,
+         win=(1, 2, 2), shift=(0, 0, 0), scale=0.125):
+    # Fake, never-dereferenced device addresses: every case below must be
+    # rejected by host-side validation before anything touches the GPU.
+    return lib.basa_swattn_fwd(ctypes.c_void_p(q), ctypes.c_void_p(k), ctypes.c_void_p(v),
+                               ctypes.c_void_p(out), B, heads, *grid, d, I3(*win), I3(*shift),
+                               ctypes.c_float(scale), None)
+
+
+def test_argument_errors_are_caught_on_the_host(lib):
+    big = 1 << 30
+    assert _fwd(lib, q=0) == sw.BASA_ERR_INVALID_ARG
+    assert _fwd(lib, out=0) == sw.BASA_ERR_INVALID_ARG
+    assert _fwd(lib, B=0, out=big) == sw.BASA_ERR_INVALID_ARG
+    assert _fwd(lib, heads=-1, out=big) == sw.BASA_ERR_INVALID_ARG
+    assert _fwd(lib, grid=(1, 0, 4), out=big) == sw.BASA_ERR_INVALID_ARG
+    assert _fwd(lib, win=(1, 5, 2), out=big) == sw.BASA_ERR_INVALID_ARG
+    assert _fwd(lib, win=(0, 2, 2), out=big) == sw.BASA_ERR_INVALID_ARG
+    assert _fwd(lib, scale=float("nan"), out=big) == sw.BASA_ERR_INVALID_ARG
+    assert _fwd(lib, scale=float("inf"), out=big) == sw.BASA_ERR_INVALID_ARG
+    assert _fwd(lib, d=96, out=big) == sw.BASA_ERR_UNSUPPORTED
+    assert _fwd(lib, d=256, out=big) == sw.BASA_ERR_UNSUPPORTED
+    assert _fwd(lib, grid=(1, 1 << 16, 1 << 16), win=(1, 1, 1), out=big) == sw.BASA_ERR_UNSUPPORTED
+    assert _fwd(lib, q=24, out=big) == sw.BASA_ERR_ALIGNMENT
+    assert _fwd(lib, out=big + 8) == sw.BASA_ERR_ALIGNMENT
+    # out overlapping an input (4x4 grid, d=64: 2 KB per tensor)
+    assert _fwd(lib, q=big, k=2 * big, v=3 * big, out=big + 1024) == sw.BASA_ERR_ALIAS
+
+
+def test_strerror_covers_every_code(lib):
+    for code in (0, -1, -2, -3, -4, -5, -6):
+        assert sw.strerror(code) != "unknown error"
+    assert sw.strerror(12345) == "unknown error"
+
+
+def test_python_binding_rejects_non_cuda_tensors(lib):
+    import torch
+    q = torch.zeros(1, 16, 1, 64, dtype=torch.bfloat16)
+    with pytest.raises(TypeError):
+        sw.swattn_fwd(q, q, q, (1, 4, 4), (1, 2, 2), (0, 0, 0))

@@ -1,0 +1,194 @@
+"""GPU parity: the sm_100a kernel against the fp64 oracle, through the C ABI.
+
+Tolerances (bf16 inputs, fp32 accumulation, P and the output rounded to bf16):
+max-abs error <= 2e-2 and relative L2 error <= 5e-3 against the oracle, over
+every compared element.  Index maps must match exactly.
+
+Small cases compare every output element; the full-size workloads compare
+sampled rows that the oracle computes one by one, in the same launch
+configuration the benchmark times.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import shifted_window_attention_swattn_b200 as sw
+from shifted_window_attention_swattn_b200.inputs import WORKLOADS, make_custom, make_qkv
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS = 2e-2
+REL_L2 = 5e-3
+
+
+def _check(got, ref, what=""):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert np.isfinite(got).all(), f"{what}: non-finite output"
+    err = np.abs(got - ref)
+    rel = np.linalg.norm((got - ref).ravel()) / max(np.linalg.norm(ref.ravel()), 1e-30)
+    assert err.max() <= MAX_ABS and rel <= REL_L2, f"{what}: max_abs={err.max():.3e} rel_l2={rel:.3e}"
+    return err.max(), rel
+
+
+def _run_gpu(q, k, v, grid, win, shift, scale):
+    dev = torch.device("cuda:0")
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    out = sw.swattn_fwd(qd, kd, vd, grid, win, shift, scale)
+    assert sw.last_device_error() == sw.BASA_OK
+    return out
+
+
+def _full_compare(B, heads, d, grid, win, shift, scale=None, seed=0, dist="normal"):
+    T, H, W = grid
+    q, k, v = make_custom(B, heads, d, T, H, W, seed, dist=dist)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    out = _run_gpu(q, k, v, grid, win, shift, scale).float().cpu().numpy()
+    ref = oracle.swattn_fwd(q, k, v, B, heads, T, H, W, d, win, shift, scale)
+    return _check(out, ref, f"grid={grid} win={win} shift={shift} d={d}")
+
+
+# ---------------------------------------------------------------- index maps
+
+@pytest.mark.parametrize("wl", WORKLOADS, ids=lambda w: w.name)
+def test_device_index_map_exact_on_workloads(wl):
+    for shift in wl.shifts:
+        got = sw.index_map(wl.grid, wl.win, shift).cpu().numpy()
+        ref, _ = oracle.index_map(*wl.grid, wl.win, shift)
+        assert np.array_equal(got, ref), shift
+
+
+@pytest.mark.parametrize("grid,win,shift", [
+    ((3, 1, 5), (2, 1, 2), (1, 0, 2)),
+    ((5, 9, 11), (2, 4, 5), (1, 7, -3)),
+    ((1, 20, 28), (1, 7, 9), (0, 3, 5)),
+])
+def test_device_index_map_exact_ragged(grid, win, shift):
+    got = sw.index_map(grid, win, shift).cpu().numpy()
+    ref, _ = oracle.index_map(*grid, win, shift)
+    assert np.array_equal(got, ref)
+
+
+# ---------------------------------------------------------------- small, every element
+
+@pytest.mark.parametrize("shift", [(0, 0, 0), (0, 4, 4)])
+def test_tiny_2d_workload(shift):
+    wl = WORKLOADS[0]
+    q, k, v = make_qkv(wl)
+    out = _run_gpu(q, k, v, wl.grid, wl.win, shift, wl.scale).float().cpu().numpy()
+    ref = oracle.swattn_fwd(q, k, v, wl.B, wl.heads, *wl.grid, wl.d, wl.win, shift, wl.scale)
+    _check(out, ref, f"tiny shift={shift}")
+
+
+@pytest.mark.parametrize("B,heads,d,grid,win,shift", [
+    (2, 3, 128, (1, 20, 28), (1, 7, 9), (0, 3, 5)),      # n_w = 63, truncated windows
+    (1, 2, 64, (5, 9, 11), (2, 4, 5), (1, 7, -3)),       # 3D, truncation on every axis
+    (1, 2, 128, (1, 24, 24), (1, 12, 13), (0, 6, 11)),   # n_w = 156: two ragged tiles
+    (1, 2, 128, (2, 16, 20), (2, 16, 10), (1, 8, 5)),    # n_w = 320: tiles 128+128+64
+    (1, 1, 128, (1, 4, 300), (1, 1, 300), (0, 1, 77)),   # 300-token row windows
+    (1, 2, 64, (1, 16, 16), (1, 8, 16), (0, 3, 9)),      # exactly 128 tokens
+    (1, 2, 128, (1, 3, 43), (1, 3, 43), (0, 1, 20)),     # 129 tokens
+    (3, 1, 64, (2, 6, 6), (1, 3, 3), (1, 1, 2)),         # B = 3
+    (1, 4, 128, (3, 10, 13), (3, 5, 13), (2, 4, 6)),     # 195 tokens, 3D
+])
+def test_ragged_and_edge_shapes(B, heads, d, grid, win, shift):
+    _full_compare(B, heads, d, grid, win, shift, seed=B * 100 + d)
+
+
+def test_full_attention_mode_tiny():
+    wl = WORKLOADS[0]
+    _full_compare(1, 2, 64, wl.grid, wl.grid, (0, 0, 0), seed=3)
+
+
+def test_sharp_softmax_exercises_rescaling():
+    # scale 1 with d = 128 gives logits of std ~11: the running max moves a lot.
+    _full_compare(1, 2, 128, (1, 24, 24), (1, 12, 12), (0, 6, 6), scale=1.0, seed=21)
+
+
+def test_uniform_inputs():
+    _full_compare(1, 2, 128, (2, 12, 12), (2, 6, 12), (1, 3, 5), seed=22, dist="uniform")
+
+
+def test_single_token_windows_return_v():
+    T, H, W = 2, 3, 8
+    q, k, v = make_custom(1, 2, 64, T, H, W, 5)
+    out = _run_gpu(q, k, v, (T, H, W), (1, 1, 1), (1, 2, 3), 0.125)
+    assert torch.equal(out.cpu(), v)
+
+
+def test_scale_zero_gives_window_mean():
+    _full_compare(1, 2, 128, (1, 12, 20), (1, 6, 10), (0, 2, 7), scale=0.0, seed=23)
+
+
+def test_shift_by_grid_extent_matches_reduced_shift():
+    T, H, W = 1, 16, 16
+    q, k, v = make_custom(1, 2, 128, T, H, W, 7)
+    a = _run_gpu(q, k, v, (T, H, W), (1, 8, 8), (0, 3, 5), 0.09)
+    b = _run_gpu(q, k, v, (T, H, W), (1, 8, 8), (5, 3 - 2 * H, 5 + W), 0.09)
+    assert torch.equal(a, b)
+
+
+def test_repeated_calls_are_deterministic():
+    T, H, W = 1, 32, 32
+    q, k, v = make_custom(1, 4, 128, T, H, W, 8)
+    a = _run_gpu(q, k, v, (T, H, W), (1, 16, 16), (0, 8, 8), 0.09)
+    b = _run_gpu(q, k, v, (T, H, W), (1, 16, 16), (0, 8, 8), 0.09)
+    assert torch.equal(a, b)
+
+
+def test_host_buffer_entry_matches_device_entry():
+    T, H, W = 1, 16, 32
+    q, k, v = make_custom(1, 2, 128, T, H, W, 9)
+    dev = _run_gpu(q, k, v, (T, H, W), (1, 8, 16), (0, 4, 8), 0.09).cpu()
+    host = sw.swattn_fwd_from_host(q.pin_memory(), k.pin_memory(), v.pin_memory(), (T, H, W),
+                                   (1, 8, 16), (0, 4, 8), 0.09)
+    assert torch.equal(dev, host)
+
+
+# ---------------------------------------------------------------- full-size workloads, sampled rows
+
+def _sample_triples(wl, shift, n_random, rng):
+    """Random (b, token, head) triples plus every query of one whole window."""
+    tri = np.stack([rng.integers(0, wl.B, n_random), rng.integers(0, wl.N, n_random),
+                    rng.integers(0, wl.heads, n_random)], axis=1)
+    tos, cnt = oracle.index_map(*wl.grid, wl.win, shift)
+    wid = int(rng.integers(0, tos.shape[0]))
+    toks = tos[wid, :cnt[wid]]
+    whole = np.stack([np.zeros_like(toks), toks, np.full_like(toks, wl.heads - 1)], axis=1)
+    return np.concatenate([tri, whole]).astype(np.int64)
+
+
+@pytest.mark.parametrize("wl", WORKLOADS[1:], ids=lambda w: w.name)
+def test_full_size_workloads_sampled(wl):
+    q, k, v = make_qkv(wl)
+    dev = torch.device("cuda:0")
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    rng = np.random.default_rng(wl.seed)
+    for shift in wl.shifts:
+        out = sw.swattn_fwd(qd, kd, vd, wl.grid, wl.win, shift, wl.scale)
+        assert sw.last_device_error() == sw.BASA_OK
+        tri = _sample_triples(wl, shift, 1500, rng)
+        ref = oracle.swattn_rows(q, k, v, wl.B, wl.heads, *wl.grid, wl.d, wl.win, shift,
+                                 wl.scale, tri)
+        got = out[tri[:, 0], tri[:, 1], tri[:, 2]].float().cpu().numpy()
+        _check(got, ref, f"{wl.name} shift={shift}")
+        assert torch.isfinite(out).all()
+        del out
+
+
+@pytest.mark.parametrize("wl", WORKLOADS[1:2], ids=lambda w: w.name)
+def test_full_attention_mode_sampled(wl):
+    q, k, v = make_qkv(wl)
+    dev = torch.device("cuda:0")
+    out = sw.swattn_fwd(q.to(dev), k.to(dev), v.to(dev), wl.grid, wl.grid, (0, 0, 0), wl.scale)
+    assert sw.last_device_error() == sw.BASA_OK
+    rng = np.random.default_rng(99)
+    tri = np.stack([np.zeros(400, dtype=np.int64), rng.integers(0, wl.N, 400),
+                    rng.integers(0, wl.heads, 400)], axis=1)
+    ref = oracle.swattn_rows(q, k, v, wl.B, wl.heads, *wl.grid, wl.d, wl.grid, (0, 0, 0),
+                             wl.scale, tri)
+    got = out[tri[:, 0], tri[:, 1], tri[:, 2]].float().cpu().numpy()
+    _check(got, ref, "full attention")
