@@ -54,7 +54,8 @@ extern "C" {
  *   q, k, v  in : device bf16 [B, T*H*W, heads, d]
  *   out      out: device bf16 [B, T*H*W, heads, d]; must not overlap q, k or v
  *   d        64 or 128
- *   scale    softmax scale applied to Q K^T (1/sqrt(d) for standard attention)
+ *   scale    softmax scale applied to Q K^T (1/sqrt(d) for standard attention);
+ *            finite and >= 0 (a negative scale returns BASA_ERR_UNSUPPORTED)
  *
  * out[b, p, h, :] = sum_j softmax_j(scale * <q_p, k_j>) v_j over the tokens j
  * that share the (shifted) window of token p.  Accumulation is fp32; P is

@@ -46,16 +46,17 @@
 
 namespace swattn {
 
-constexpr int kThreads = 192;
-constexpr int kTile = 128;       // query rows per CTA tile = key rows per K/V tile
-constexpr int kStages = 2;       // K/V ring depth
-constexpr int kSoftmaxWarps = 4;
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
+constexpr int kThreads = 352;    // 11 warps
+constexpr int kTile = 128;       // query rows per tile = key rows per K/V tile
+constexpr int kMaxSlots = 8;     // K/V ring depth limit (tiles)
+constexpr int kProducerWarp0 = 8;  // warps 8 and 9 each load half of every tile
+constexpr int kProducers = 2;
+constexpr int kMmaWarp = 10;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0;     // S buffer b at kColS + 128 * b
-constexpr uint32_t kColO = 256;
-constexpr uint32_t kColP = 384;   // P buffer b at kColP + 64 * b
+constexpr uint32_t kColS0 = 0;   // S_0 (P_0 in its first 64 columns as bf16 pairs)
+constexpr uint32_t kColS1 = 128; // S_1 (P_1 likewise)
+constexpr uint32_t kColO0 = 256;
+constexpr uint32_t kColO1 = 384;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: O is rescaled when the max grows by > 2^8
 
 // ------------------------------------------------------------------ geometry
@@ -135,23 +136,25 @@ struct __align__(64) FwdParams {
   __nv_bfloat16* out;
   Geometry g;
   int B, heads, d;
-  int q_tiles;                  // ceil(nw_max / 128)
+  int q_pairs;                  // ceil(nw_max / 256): 256-query units per window
+  int total_units;              // B * heads * n_windows * q_pairs
+  int n_slots;                  // K/V ring depth (tiles)
   float scale_log2;             // scale * log2(e)
   unsigned long long timeout_ns;
 };
 
 struct SmemCtl {
-  uint64_t q_full;
-  uint64_t k_full[kStages];
-  uint64_t v_full[kStages];
-  uint64_t kv_empty[kStages];
-  uint64_t s_full[2];
-  uint64_t p_full[2];
-  uint64_t o_done;              // P V of every tile but the last
-  uint64_t o_final;             // P V of the last tile
-  uint64_t drained;             // every MMA of the CTA
+  uint64_t q_full[2];
+  uint64_t q_empty[2];
+  uint64_t kv_full[kMaxSlots];
+  uint64_t kv_empty[kMaxSlots];
+  uint64_t s_full[2];           // S_i = Q_i K_j^T is in TMEM
+  uint64_t p_full[2];           // P_i is in TMEM and O_i is rescaled
+  uint64_t o_final[2];          // last P V of the unit for tile i is done
+  uint64_t drained;             // every MMA of the CTA is done
   uint32_t tmem_base;
   int abort;
+  int rows[kProducers][kTile / kProducers];   // gather coordinates staged per producer warp
 };
 
 __device__ int g_device_error = 0;
@@ -165,8 +168,94 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Sm
   return false;
 }
 
-__device__ __forceinline__ int token_row(const FwdParams& p, int b, int h, int token) {
-  return (b * p.g.N + token) * p.heads + h;
+// One unit of work: up to 256 queries (two 128-row tiles) of one window of
+// one (batch item, head), attending to every key of that window.
+struct Unit {
+  int b, h;
+  int m[3], e[3];
+  int n_valid;    // tokens in the window
+  int q0;         // first query slot of tile 0
+  int nkv;        // key tiles
+  bool has_q1;    // tile 1 holds at least one query
+};
+
+// Units are numbered with the query pair fastest, then window, then
+// (batch, head), so CTAs that run at the same time share K/V in L2.
+__device__ __forceinline__ bool decode_unit(const FwdParams& p, int u, Unit& U) {
+  const int qp = u % p.q_pairs;
+  const int r = u / p.q_pairs;
+  const int win_id = r % p.g.n_windows;
+  const int bh = r / p.g.n_windows;
+  U.b = bh / p.heads;
+  U.h = bh - U.b * p.heads;
+  window_of(p.g, win_id, U.m, U.e);
+  U.n_valid = U.e[0] * U.e[1] * U.e[2];
+  U.q0 = qp * 2 * kTile;
+  if (U.q0 >= U.n_valid) return false;   // a truncated window has fewer query pairs
+  U.has_q1 = U.q0 + kTile < U.n_valid;
+  U.nkv = (U.n_valid + kTile - 1) / kTile;
+  return true;
+}
+
+__device__ __forceinline__ int unit_row(const FwdParams& p, const Unit& U, int slot) {
+  if (slot >= U.n_valid) slot = U.n_valid - 1;   // padding rows repeat the last token
+  return (U.b * p.g.N + slot_token(p.g, U.m, U.e, slot)) * p.heads + U.h;
+}
+
+__device__ __forceinline__ int kv_valid_of(const Unit& U, int j) {
+  const int left = U.n_valid - j * kTile;
+  return left < kTile ? left : kTile;
+}
+
+// S_i (+)= Q_i K^T over the head dimension: d/16 MMAs of M=128, N=n_s, K=16.
+__device__ __forceinline__ void issue_qk(uint32_t tmem_s, uint32_t q_addr, uint32_t k_addr, int d,
+                                         int n_s) {
+  const uint32_t idesc = idesc_bf16_f32(128, n_s, 0, 0);
+  for (int kk = 0; kk < d / 16; ++kk) {
+    const uint32_t off = (kk >> 2) * (kTile * 128) + (kk & 3) * 32;
+    umma_ss(tmem_s, smem_desc_sw128(q_addr + off, 16, 1024), smem_desc_sw128(k_addr + off, 16, 1024),
+            idesc, kk > 0 ? 1u : 0u);
+  }
+}
+
+// O_i (+)= P_i V over the keys of one tile: P_i (bf16) sits in TMEM at tmem_p.
+__device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint32_t v_addr, int d,
+                                         int kv_valid, bool accumulate) {
+  const uint32_t idesc = idesc_bf16_f32(128, d, 0, 1);
+  const int ksteps = (kv_valid + 15) >> 4;
+  for (int kk = 0; kk < ksteps; ++kk)
+    umma_ts(tmem_o, tmem_p + kk * 8, smem_desc_sw128(v_addr + kk * 2048, kTile * 128, 1024), idesc,
+            (accumulate || kk > 0) ? 1u : 0u);
+}
+
+// P = exp2(x * scale_log2 - m) for one S row held in registers, packed to
+// bf16 pairs and stored over the front of the S row in TMEM; returns the row
+// sum of the fp32 values.  kPartial: columns >= kv_valid are padding keys and
+// get P = 0.
+template <bool kPartial>
+__device__ __forceinline__ float softmax_to_p(const float (&x)[kTile], int nchunks, int kv_valid,
+                                              float sl2, float neg_m, uint32_t tS) {
+  float rowsum = 0.0f;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    if (c < nchunks) {
+      uint32_t pk[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int col = c * 32 + 2 * i;
+        float p0 = ex2_approx(fmaf(x[col], sl2, neg_m));
+        float p1 = ex2_approx(fmaf(x[col + 1], sl2, neg_m));
+        if (kPartial) {
+          p0 = col < kv_valid ? p0 : 0.0f;
+          p1 = col + 1 < kv_valid ? p1 : 0.0f;
+        }
+        rowsum += p0 + p1;
+        pk[i] = pack_bf16x2(p0, p1);
+      }
+      tmem_st16(tS + c * 16, pk);   // P overwrites the front of the S row
+    }
+  }
+  return rowsum;
 }
 
 __global__ void __launch_bounds__(kThreads, 1) swattn_fwd_kernel(const __grid_constant__ FwdParams p) {
@@ -175,47 +264,31 @@ __global__ void __launch_bounds__(kThreads, 1) swattn_fwd_kernel(const __grid_co
                                              ~static_cast<uintptr_t>(1023));
   const int d = p.d;
   const int tile_bytes = kTile * d * 2;
-  uint8_t* sQ = smem;
-  uint8_t* sK = sQ + tile_bytes;
-  uint8_t* sV = sK + kStages * tile_bytes;
-  SmemCtl* ctl = reinterpret_cast<SmemCtl*>(sV + kStages * tile_bytes);
-
-  // ---- work unit: (batch*head, window, query tile), query tile fastest
-  int unit = blockIdx.x;
-  const int qt = unit % p.q_tiles;
-  unit /= p.q_tiles;
-  const int win_id = unit % p.g.n_windows;
-  const int bh = unit / p.g.n_windows;
-  const int b = bh / p.heads;
-  const int h = bh % p.heads;
-  int m[3], e[3];
-  window_of(p.g, win_id, m, e);
-  const int n_valid = e[0] * e[1] * e[2];
-  const int q0 = qt * kTile;
-  if (q0 >= n_valid) return;   // a truncated window has fewer query tiles (CTA-uniform)
-  const int nkv = (n_valid + kTile - 1) / kTile;
+  const int n_slots = p.n_slots;
+  uint8_t* sQ = smem;                           // two query tiles
+  uint8_t* sRing = sQ + 2 * tile_bytes;         // K/V ring
+  SmemCtl* ctl = reinterpret_cast<SmemCtl*>(sRing + n_slots * tile_bytes);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    mbar_init(&ctl->q_full, 1);
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&ctl->k_full[s], 1);
-      mbar_init(&ctl->v_full[s], 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&ctl->q_full[i], kProducers);
+      mbar_init(&ctl->q_empty[i], 1);
+      mbar_init(&ctl->s_full[i], 1);
+      mbar_init(&ctl->p_full[i], 4);
+      mbar_init(&ctl->o_final[i], 1);
+    }
+    for (int s = 0; s < n_slots; ++s) {
+      mbar_init(&ctl->kv_full[s], kProducers);
       mbar_init(&ctl->kv_empty[s], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&ctl->s_full[i], 1);
-      mbar_init(&ctl->p_full[i], kSoftmaxWarps);
-    }
-    mbar_init(&ctl->o_done, 1);
-    mbar_init(&ctl->o_final, 1);
     mbar_init(&ctl->drained, 1);
     ctl->abort = 0;
     fence_barrier_init();
   }
-  if (warp == kProducerWarp && lane == 0) {
+  if (warp == kProducerWarp0 && lane == 0) {
     prefetch_tensormap(&p.tq);
     prefetch_tensormap(&p.tk);
     prefetch_tensormap(&p.tv);
@@ -229,109 +302,145 @@ __global__ void __launch_bounds__(kThreads, 1) swattn_fwd_kernel(const __grid_co
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
 
-  if (warp == kProducerWarp) {
-    // ================================================================ producer
-    const int ncb = d / 64;   // 64-column (128-byte) blocks per row
-    int last_tile_in_stage[kStages];
-    for (int s = 0; s < kStages; ++s) last_tile_in_stage[s] = -1;
-    int r[4];
-    // Q tile: slots q0 .. q0+127, rows past the window repeat its last token
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      int s = q0 + 4 * lane + i;
-      if (s >= n_valid) s = n_valid - 1;
-      r[i] = token_row(p, b, h, slot_token(p.g, m, e, s));
-    }
-    if (lane == 0) mbar_arrive_expect_tx(&ctl->q_full, tile_bytes);
-    __syncwarp();
-    for (int c = 0; c < ncb; ++c)
-      tma_gather4(&p.tq, &ctl->q_full, sQ + c * (kTile * 128) + lane * 512, c * 64, r[0], r[1],
-                  r[2], r[3]);
-    for (int j = 0; j < nkv; ++j) {
-      const int s = j % kStages;
-      if (j >= kStages) {
-        bool ok = wait_or_abort(&ctl->kv_empty[s], ((j / kStages) - 1) & 1, ctl, p.timeout_ns);
-        if (!__all_sync(0xffffffffu, ok)) break;
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        int sl = j * kTile + 4 * lane + i;
-        if (sl >= n_valid) sl = n_valid - 1;
-        r[i] = token_row(p, b, h, slot_token(p.g, m, e, sl));
-      }
-      uint8_t* dk = sK + s * tile_bytes;
-      uint8_t* dv = sV + s * tile_bytes;
-      if (lane == 0) mbar_arrive_expect_tx(&ctl->k_full[s], tile_bytes);
+  if (warp >= kProducerWarp0 && warp < kProducerWarp0 + kProducers) {
+    // ================================================================ TMA producers
+    // Each producer warp loads rows [pw*64, pw*64+64) of every tile.  All lanes
+    // compute gather coordinates into shared memory; the warp then walks them
+    // with warp-uniform control flow and one elected lane issues each load.
+    const int pw = warp - kProducerWarp0;
+    constexpr int kRowsPer = kTile / kProducers;
+    const int ncb = d / 64;   // 128-byte column blocks per row
+    const uint32_t half_bytes = tile_bytes / kProducers;
+    int* rows = ctl->rows[pw];
+    const int4* rows4 = reinterpret_cast<const int4*>(rows);
+    uint32_t q_use[2] = {0, 0};
+    uint32_t ld = 0;          // loads issued into the ring
+    bool ok = true;
+    auto stage_rows = [&](const Unit& U, int slot0) {
       __syncwarp();
-      for (int c = 0; c < ncb; ++c)
-        tma_gather4(&p.tk, &ctl->k_full[s], dk + c * (kTile * 128) + lane * 512, c * 64, r[0],
-                    r[1], r[2], r[3]);
-      if (lane == 0) mbar_arrive_expect_tx(&ctl->v_full[s], tile_bytes);
+      for (int x = lane; x < kRowsPer; x += 32) rows[x] = unit_row(p, U, slot0 + pw * kRowsPer + x);
       __syncwarp();
-      for (int c = 0; c < ncb; ++c)
-        tma_gather4(&p.tv, &ctl->v_full[s], dv + c * (kTile * 128) + lane * 512, c * 64, r[0],
-                    r[1], r[2], r[3]);
-      last_tile_in_stage[s] = j;
-    }
-    // Drain: every load this warp issued has landed before the CTA can exit.
-    // (In the normal flow these phases are long complete and return at once.)
-    mbar_wait_bounded(&ctl->q_full, 0, p.timeout_ns);
-    for (int s = 0; s < kStages; ++s) {
-      const int j = last_tile_in_stage[s];
-      if (j >= 0) {
-        mbar_wait_bounded(&ctl->k_full[s], (j / kStages) & 1, p.timeout_ns);
-        mbar_wait_bounded(&ctl->v_full[s], (j / kStages) & 1, p.timeout_ns);
+    };
+    auto issue = [&](const CUtensorMap* map, uint64_t* bar, uint8_t* tile) {
+      if (elect_one()) mbar_arrive_expect_tx(bar, half_bytes);
+      __syncwarp();
+      uint8_t* dst = tile + pw * kRowsPer * 128;
+      for (int g = 0; g < kRowsPer / 4; ++g) {
+        const int4 r = rows4[g];
+        if (elect_one())
+          for (int c = 0; c < ncb; ++c)
+            tma_gather4(map, bar, dst + c * (kTile * 128) + g * 512, c * 64, r.x, r.y, r.z, r.w);
+        __syncwarp();
+      }
+    };
+    for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
+      Unit U;
+      if (!decode_unit(p, u, U)) continue;
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        if (i == 1 && !U.has_q1) break;
+        if (q_use[i] > 0) {
+          ok = __all_sync(0xffffffffu,
+                          wait_or_abort(&ctl->q_empty[i], (q_use[i] - 1) & 1, ctl, p.timeout_ns));
+          if (!ok) break;
+        }
+        stage_rows(U, U.q0 + i * kTile);
+        issue(&p.tq, &ctl->q_full[i], sQ + i * tile_bytes);
+        ++q_use[i];
+      }
+      for (int j = 0; ok && j < U.nkv; ++j) {
+        stage_rows(U, j * kTile);
+        for (int kv = 0; kv < 2; ++kv) {
+          const int slot = ld % n_slots;
+          const uint32_t use = ld / n_slots;
+          if (use > 0) {
+            ok = __all_sync(0xffffffffu,
+                            wait_or_abort(&ctl->kv_empty[slot], (use - 1) & 1, ctl, p.timeout_ns));
+            if (!ok) break;
+          }
+          issue(kv == 0 ? &p.tk : &p.tv, &ctl->kv_full[slot], sRing + slot * tile_bytes);
+          ++ld;
+        }
       }
     }
+    // Drain: every load issued has landed before the CTA can exit.  In the
+    // normal flow these phases completed long ago and the waits return at once.
+    for (int i = 0; i < 2; ++i)
+      if (q_use[i] > 0) mbar_wait_bounded(&ctl->q_full[i], (q_use[i] - 1) & 1, p.timeout_ns);
+    for (uint32_t x = (ld > static_cast<uint32_t>(n_slots) ? ld - n_slots : 0); x < ld; ++x)
+      mbar_wait_bounded(&ctl->kv_full[x % n_slots], (x / n_slots) & 1, p.timeout_ns);
   } else if (warp == kMmaWarp) {
     // ================================================================ MMA issuer
     if (lane == 0) {
-      const uint32_t q_addr = smem_u32(sQ);
-      const uint32_t k_addr = smem_u32(sK);
-      const uint32_t v_addr = smem_u32(sV);
-      const uint32_t idesc_pv = idesc_bf16_f32(128, d, 0, 1);
-      const int ksteps_qk = d / 16;
-      bool ok = wait_or_abort(&ctl->q_full, 0, ctl, p.timeout_ns);
-      for (int j = 0; ok && j <= nkv; ++j) {
-        if (j < nkv) {
-          const int s = j % kStages;
-          const int bb = j & 1;
-          ok = wait_or_abort(&ctl->k_full[s], (j / kStages) & 1, ctl, p.timeout_ns);
-          if (!ok) break;
-          tc_fence_after();
-          int kv_valid = n_valid - j * kTile;
-          if (kv_valid > kTile) kv_valid = kTile;
-          const int n_s = (kv_valid + 15) & ~15;
-          const uint32_t idesc_s = idesc_bf16_f32(128, n_s, 0, 0);
-          const uint32_t kbase = k_addr + s * tile_bytes;
-          for (int kk = 0; kk < ksteps_qk; ++kk) {
-            const uint32_t off = (kk >> 2) * (kTile * 128) + (kk & 3) * 32;
-            umma_ss(tmem + kColS + 128u * bb, smem_desc_sw128(q_addr + off, 16, 1024),
-                    smem_desc_sw128(kbase + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+      const uint32_t q_addr[2] = {smem_u32(sQ), smem_u32(sQ + tile_bytes)};
+      const uint32_t ring_addr = smem_u32(sRing);
+      const uint32_t tS[2] = {tmem + kColS0, tmem + kColS1};
+      const uint32_t tO[2] = {tmem + kColO0, tmem + kColO1};
+      uint32_t q_use[2] = {0, 0};
+      uint32_t p_use[2] = {0, 0};
+      uint32_t ld = 0;        // ring tiles consumed
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
+        Unit U;
+        if (!decode_unit(p, u, U)) continue;
+        const int nq = U.has_q1 ? 2 : 1;
+#pragma unroll
+        for (int i = 0; i < 2; ++i)
+          if (ok && i < nq) ok = wait_or_abort(&ctl->q_full[i], q_use[i] & 1, ctl, p.timeout_ns);
+        if (!ok) break;
+        // K_0 -> S_i(0)
+        int slot_k = ld % n_slots;
+        ok = wait_or_abort(&ctl->kv_full[slot_k], (ld / n_slots) & 1, ctl, p.timeout_ns);
+        if (!ok) break;
+        ++ld;
+        tc_fence_after();
+        {
+          const int n_s = (kv_valid_of(U, 0) + 15) & ~15;
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            if (i >= nq) break;
+            issue_qk(tS[i], q_addr[i], ring_addr + slot_k * tile_bytes, d, n_s);
+            umma_commit(&ctl->s_full[i]);
+            if (U.nkv == 1) umma_commit(&ctl->q_empty[i]);
           }
-          umma_commit(&ctl->s_full[bb]);
+          umma_commit(&ctl->kv_empty[slot_k]);
         }
-        if (j >= 1) {
-          const int jp = j - 1;
-          const int sp = jp % kStages;
-          const int bp = jp & 1;
-          ok = wait_or_abort(&ctl->p_full[bp], (jp >> 1) & 1, ctl, p.timeout_ns);
+        for (int j = 0; j < U.nkv; ++j) {
+          const int slot_v = ld % n_slots;
+          ok = wait_or_abort(&ctl->kv_full[slot_v], (ld / n_slots) & 1, ctl, p.timeout_ns);
           if (!ok) break;
-          ok = wait_or_abort(&ctl->v_full[sp], (jp / kStages) & 1, ctl, p.timeout_ns);
-          if (!ok) break;
-          tc_fence_after();
-          int kv_valid = n_valid - jp * kTile;
-          if (kv_valid > kTile) kv_valid = kTile;
-          const int ksteps = (kv_valid + 15) >> 4;
-          const uint32_t vbase = v_addr + sp * tile_bytes;
-          for (int kk = 0; kk < ksteps; ++kk) {
-            umma_ts(tmem + kColO, tmem + kColP + 64u * bp + kk * 8,
-                    smem_desc_sw128(vbase + kk * 2048, kTile * 128, 1024), idesc_pv,
-                    (jp > 0 || kk > 0) ? 1u : 0u);
+          ++ld;
+          const bool more = j + 1 < U.nkv;
+          const int kvv = kv_valid_of(U, j);
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            if (i >= nq) break;
+            ok = wait_or_abort(&ctl->p_full[i], p_use[i] & 1, ctl, p.timeout_ns);
+            if (!ok) break;
+            ++p_use[i];
+            tc_fence_after();
+            issue_pv(tO[i], tS[i], ring_addr + slot_v * tile_bytes, d, kvv, j > 0);
+            if (!more) umma_commit(&ctl->o_final[i]);
+            if (i == nq - 1) umma_commit(&ctl->kv_empty[slot_v]);
+            if (more) {
+              if (i == 0) {
+                slot_k = ld % n_slots;
+                ok = wait_or_abort(&ctl->kv_full[slot_k], (ld / n_slots) & 1, ctl, p.timeout_ns);
+                if (!ok) break;
+                ++ld;
+                tc_fence_after();
+              }
+              const int n_s = (kv_valid_of(U, j + 1) + 15) & ~15;
+              issue_qk(tS[i], q_addr[i], ring_addr + slot_k * tile_bytes, d, n_s);
+              umma_commit(&ctl->s_full[i]);
+              if (j + 1 == U.nkv - 1) umma_commit(&ctl->q_empty[i]);
+              if (i == nq - 1) umma_commit(&ctl->kv_empty[slot_k]);
+            }
           }
-          umma_commit(&ctl->kv_empty[sp]);
-          umma_commit(jp == nkv - 1 ? &ctl->o_final : &ctl->o_done);
+          if (!ok) break;
         }
+        ++q_use[0];
+        if (nq == 2) ++q_use[1];
       }
       // Drain every MMA this thread issued before TMEM is released.
       umma_commit(&ctl->drained);
@@ -339,108 +448,99 @@ __global__ void __launch_bounds__(kThreads, 1) swattn_fwd_kernel(const __grid_co
     }
     __syncwarp();
   } else {
-    // ================================================================ softmax
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    // ================================================================ softmax (+ correction, epilogue)
+    const int wg = warp >> 2;                         // query tile 0 or 1
+    const int row = threadIdx.x & 127;                // query row within the tile
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + (wg ? kColS1 : kColS0) + lane_off;
+    const uint32_t tO = tmem + (wg ? kColO1 : kColO0) + lane_off;
     const float sl2 = p.scale_log2;
-    float m_run = -INFINITY;
-    float l_run = 0.0f;
+    uint32_t s_use = 0, of_use = 0;
     bool ok = true;
-    for (int j = 0; j < nkv; ++j) {
-      const int bb = j & 1;
-      ok = wait_or_abort(&ctl->s_full[bb], (j >> 1) & 1, ctl, p.timeout_ns);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      tc_fence_after();
-      int kv_valid = n_valid - j * kTile;
-      if (kv_valid > kTile) kv_valid = kTile;
-      const int nchunks = (kv_valid + 31) >> 5;
-
-      float x[kTile];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        if (c < nchunks) {
-          uint32_t r[32];
-          tmem_ld32(tmem + kColS + 128u * bb + lane_off + c * 32, r);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) x[c * 32 + i] = __uint_as_float(r[i]);
-        }
-      }
-      tmem_wait_ld();
-      float mx = -INFINITY;
-#pragma unroll
-      for (int i = 0; i < kTile; ++i) {
-        x[i] = (i < kv_valid) ? x[i] * sl2 : -INFINITY;
-        mx = fmaxf(mx, x[i]);
-      }
-      const float m_new = fmaxf(m_run, mx);
-      const bool need = m_new > m_run + kRescaleThreshold;
-      float alpha = 1.0f;
-      if (need) {
-        alpha = ex2_approx(m_run - m_new);
-        m_run = m_new;
-      }
-      float rowsum = 0.0f;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        if (c < nchunks) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float p0 = ex2_approx(x[c * 32 + 2 * i] - m_run);
-            const float p1 = ex2_approx(x[c * 32 + 2 * i + 1] - m_run);
-            rowsum += p0 + p1;
-            pk[i] = pack_bf16x2(p0, p1);
-          }
-          tmem_st16(tmem + kColP + 64u * bb + lane_off + c * 16, pk);
-        }
-      }
-      l_run = l_run * alpha + rowsum;
-      if (j >= 1 && __any_sync(0xffffffffu, need)) {
-        // O holds P V of tiles 0..j-1 relative to the old max: wait for the
-        // last of them to finish, then scale the row by alpha.
-        bool ok2 = wait_or_abort(&ctl->o_done, (j - 1) & 1, ctl, p.timeout_ns);
-        ok2 = __all_sync(0xffffffffu, ok2);
-        if (!ok2) {
-          ok = false;
-          break;
-        }
+    for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
+      Unit U;
+      if (!decode_unit(p, u, U)) continue;
+      if (wg == 1 && !U.has_q1) continue;
+      float m_run = -INFINITY;   // running max of scale*log2(e)*S (possibly stale by < 8)
+      float l_run = 0.0f;        // running sum of exp2(x - m_run)
+      for (int j = 0; j < U.nkv; ++j) {
+        ok = __all_sync(0xffffffffu, wait_or_abort(&ctl->s_full[wg], s_use & 1, ctl, p.timeout_ns));
+        if (!ok) break;
+        ++s_use;
         tc_fence_after();
-        for (int c = 0; c < d / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tmem + kColO + lane_off + c * 32, r);
-          tmem_wait_ld();
+        const int kvv = kv_valid_of(U, j);
+        const int nchunks = (kvv + 31) >> 5;
+        float x[kTile];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-          tmem_st32(tmem + kColO + lane_off + c * 32, r);
+        for (int c = 0; c < 4; ++c) {
+          if (c < nchunks) {
+            uint32_t r[32];
+            tmem_ld32(tS + c * 32, r);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) x[c * 32 + i] = __uint_as_float(r[i]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) x[c * 32 + i] = -INFINITY;
+          }
         }
+        tmem_wait_ld();
+        if (kvv < kTile) {
+#pragma unroll
+          for (int i = 0; i < kTile; ++i)
+            if (i >= kvv) x[i] = -INFINITY;
+        }
+        float mx = x[0];
+#pragma unroll
+        for (int i = 1; i < kTile; ++i) mx = fmaxf(mx, x[i]);
+        const float m_new = fmaxf(m_run, mx * sl2);
+        const bool need = m_new > m_run + kRescaleThreshold;
+        float alpha = 1.0f;
+        if (need) {
+          alpha = ex2_approx(m_run - m_new);
+          m_run = m_new;
+        }
+        const float neg_m = -m_run;
+        const float rowsum = kvv < kTile ? softmax_to_p<true>(x, nchunks, kvv, sl2, neg_m, tS)
+                                         : softmax_to_p<false>(x, nchunks, kvv, sl2, neg_m, tS);
+        l_run = l_run * alpha + rowsum;
+        if (j > 0 && __any_sync(0xffffffffu, need)) {
+          // O_i holds P V of tiles 0..j-1 (complete: S_i(j) was issued after
+          // them) relative to the old max; rescale the row by alpha.  Done
+          // after P so that the S row is no longer live in registers.
+          for (int c = 0; c < d / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld32(tO + c * 32, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+            tmem_st32(tO + c * 32, r);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl->p_full[wg]);
       }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ctl->p_full[bb]);
-    }
-    // ---- epilogue: O / l, bf16, stored at the row the query came from
-    if (ok) {
-      ok = wait_or_abort(&ctl->o_final, 0, ctl, p.timeout_ns);
-      ok = __all_sync(0xffffffffu, ok);
-    }
-    if (ok) {
+      if (!ok) break;
+      // ---- epilogue: O / l in bf16, stored at the row the query came from
+      ok = __all_sync(0xffffffffu, wait_or_abort(&ctl->o_final[wg], of_use & 1, ctl, p.timeout_ns));
+      if (!ok) break;
+      ++of_use;
       tc_fence_after();
-      const int slot = q0 + static_cast<int>(threadIdx.x);
-      const bool valid = slot < n_valid;
+      const int slot = U.q0 + wg * kTile + row;
+      const bool valid = slot < U.n_valid;
       __nv_bfloat16* dst = nullptr;
       if (valid)
-        dst = p.out + static_cast<size_t>(token_row(p, b, h, slot_token(p.g, m, e, slot))) * d;
+        dst = p.out + static_cast<size_t>(unit_row(p, U, slot)) * d;
       const float inv_l = 1.0f / l_run;
       for (int c = 0; c < d / 32; ++c) {
         uint32_t r[32];
-        tmem_ld32(tmem + kColO + lane_off + c * 32, r);
+        tmem_ld32(tO + c * 32, r);
         tmem_wait_ld();
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i)
-          pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * inv_l,
-                              __uint_as_float(r[2 * i + 1]) * inv_l);
+          pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * inv_l, __uint_as_float(r[2 * i + 1]) * inv_l);
         if (valid) {
           uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
 #pragma unroll
@@ -448,6 +548,7 @@ __global__ void __launch_bounds__(kThreads, 1) swattn_fwd_kernel(const __grid_co
             d4[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
         }
       }
+      tc_fence_before();   // O_i reads are ordered before the next unit's P V (via p_full)
     }
   }
 
@@ -456,6 +557,421 @@ __global__ void __launch_bounds__(kThreads, 1) swattn_fwd_kernel(const __grid_co
   if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ============================================================================
+// CTA-pair kernel (head dim 128): the same computation with tcgen05 MMAs of
+// M = 256 split over the two CTAs of a cluster.  Each CTA owns 128 query rows
+// of every tile and half of every K/V tile (half of the keys of K, half of the
+// head dimension of V), so each SM loads half the K/V bytes of the one-CTA
+// kernel and each MMA reads half of its B operand from each SM.
+//
+// Per CTA: warps 0-7 softmax (two query tiles, ping-pong), warps 8-10 TMA
+// producers, warp 11 TMEM owner; in the leader CTA (rank 0) warp 11 also
+// issues every MMA of the pair.  Barriers that gate MMAs (q_full, kv_full,
+// p_full) live in the leader and count both CTAs; barriers that MMAs signal
+// (s_full, o_final, q_empty, kv_empty) are arrived on in both CTAs.
+// ============================================================================
+
+constexpr int kPairThreads = 384;   // 12 warps
+constexpr int kPairProducer0 = 8;
+constexpr int kPairProducers = 3;
+constexpr int kPairMmaWarp = 11;
+constexpr int kPairHalfTileBytes = 16384;   // a K half (64 keys x 128) or V half (128 keys x 64)
+constexpr int kPairMaxSlots = 12;
+
+struct __align__(64) PairParams {
+  CUtensorMap tq, tk, tv;       // 2D [rows = B*N*heads, cols = 128], box {64, 1}, 128B swizzle
+  __nv_bfloat16* out;
+  Geometry g;
+  int B, heads;
+  int q_quads;                  // ceil(nw_max / 512): 512-query units per window
+  int total_units;
+  int n_slots;
+  float scale_log2;
+  unsigned long long timeout_ns;
+};
+
+struct PairCtl {
+  uint64_t q_full[2];           // leader: both CTAs' Q tile i landed
+  uint64_t q_empty[2];          // both: Q tile i may be overwritten
+  uint64_t kv_full[kPairMaxSlots];   // leader: both halves of a ring slot landed
+  uint64_t kv_empty[kPairMaxSlots];  // both: ring slot may be overwritten
+  uint64_t s_full[2];           // both: S_i in TMEM
+  uint64_t p_full[2];           // leader: P_i written (and O_i rescaled) in both CTAs
+  uint64_t o_final[2];          // both: last P V of the unit for tile i done
+  uint64_t drained;             // leader: every MMA done
+  uint32_t tmem_base;
+  int abort;
+  int rows[kPairProducers][kTile];   // gather coordinates staged per producer warp
+};
+
+__device__ __forceinline__ bool pair_wait(uint64_t* bar, uint32_t parity, PairCtl* ctl,
+                                          unsigned long long timeout_ns, bool cluster_scope) {
+  if (*reinterpret_cast<volatile int*>(&ctl->abort)) return false;
+  const bool ok = cluster_scope ? mbar_wait_bounded_cluster(bar, parity, timeout_ns)
+                                : mbar_wait_bounded(bar, parity, timeout_ns);
+  if (ok) return true;
+  *reinterpret_cast<volatile int*>(&ctl->abort) = 1;
+  atomicOr(&g_device_error, 1);
+  return false;
+}
+
+// A pair unit: up to 512 queries; tile i of CTA c holds slots q0 + 256 i + 128 c + [0, 128).
+__device__ __forceinline__ bool decode_pair_unit(const PairParams& p, int u, Unit& U) {
+  const int qp = u % p.q_quads;
+  const int r = u / p.q_quads;
+  const int win_id = r % p.g.n_windows;
+  const int bh = r / p.g.n_windows;
+  U.b = bh / p.heads;
+  U.h = bh - U.b * p.heads;
+  window_of(p.g, win_id, U.m, U.e);
+  U.n_valid = U.e[0] * U.e[1] * U.e[2];
+  U.q0 = qp * 4 * kTile;
+  if (U.q0 >= U.n_valid) return false;
+  U.has_q1 = U.q0 + 2 * kTile < U.n_valid;
+  U.nkv = (U.n_valid + kTile - 1) / kTile;
+  return true;
+}
+
+__device__ __forceinline__ int pair_row(const PairParams& p, const Unit& U, int slot) {
+  if (slot >= U.n_valid) slot = U.n_valid - 1;
+  return (U.b * p.g.N + slot_token(p.g, U.m, U.e, slot)) * p.heads + U.h;
+}
+
+// Keys of tile j used by the MMAs: all 128, or the valid keys rounded up to 32
+// for the last tile (each CTA then holds half of them).
+__device__ __forceinline__ int pair_ns(const Unit& U, int j) {
+  const int kvv = kv_valid_of(U, j);
+  return kvv == kTile ? kTile : ((kvv + 31) & ~31);
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
+    swattn_fwd_pair_kernel(const __grid_constant__ PairParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  constexpr int kQBytes = kTile * 128 * 2;
+  const int n_slots = p.n_slots;
+  uint8_t* sQ = smem;                                   // two own query tiles
+  uint8_t* sRing = sQ + 2 * kQBytes;                    // K/V half tiles
+  PairCtl* ctl = reinterpret_cast<PairCtl*>(sRing + n_slots * kPairHalfTileBytes);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int cluster_id = blockIdx.x >> 1;
+  const int n_clusters = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&ctl->q_full[i], 1);
+      mbar_init(&ctl->q_empty[i], 1);
+      mbar_init(&ctl->s_full[i], 1);
+      mbar_init(&ctl->p_full[i], 8);
+      mbar_init(&ctl->o_final[i], 1);
+    }
+    for (int s = 0; s < n_slots; ++s) {
+      mbar_init(&ctl->kv_full[s], 1);
+      mbar_init(&ctl->kv_empty[s], 1);
+    }
+    mbar_init(&ctl->drained, 1);
+    ctl->abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == kPairProducer0 && lane == 0) {
+    prefetch_tensormap(&p.tq);
+    prefetch_tensormap(&p.tk);
+    prefetch_tensormap(&p.tv);
+  }
+  if (warp == kPairMmaWarp) {
+    tmem_alloc_pair(&ctl->tmem_base, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem = ctl->tmem_base;
+
+  if (warp >= kPairProducer0 && warp < kPairProducer0 + kPairProducers) {
+    // ================================================================ TMA producers
+    // Gathers of every tile are spread over the three producer warps; each
+    // warp stages the tile's 128 row coordinates in shared memory, walks them
+    // with warp-uniform control flow, and one elected lane issues each load.
+    // Loads land in this CTA and are counted on the leader's barriers.
+    const int pw = warp - kPairProducer0;
+    int* rows = ctl->rows[pw];
+    const int4* rows4 = reinterpret_cast<const int4*>(rows);
+    uint32_t q_use[2] = {0, 0};
+    uint32_t ld = 0;
+    bool ok = true;
+    auto stage = [&](const Unit& U, int slot0) {
+      __syncwarp();
+#pragma unroll
+      for (int x = 0; x < 4; ++x) rows[lane * 4 + x] = pair_row(p, U, slot0 + lane * 4 + x);
+      __syncwarp();
+    };
+    // `count` gathers numbered 0..count-1; gather n covers row group
+    // first_group + n / nblk and column block n % nblk, at dst + (n / nblk) * 512
+    // + (n % nblk) * blk_stride, column col0 + 64 * (n % nblk).
+    auto gathers = [&](const CUtensorMap* map, uint32_t bar_leader, uint8_t* dst, int first_group,
+                       int count, int nblk, int blk_stride, int col0) {
+      for (int n = pw; n < count; n += kPairProducers) {
+        const int grp = n / nblk, blk = n - grp * nblk;
+        const int4 r = rows4[first_group + grp];
+        if (elect_one())
+          tma_gather4_pair(map, bar_leader, dst + grp * 512 + blk * blk_stride, col0 + 64 * blk, r.x,
+                           r.y, r.z, r.w);
+        __syncwarp();
+      }
+    };
+    for (int u = cluster_id; ok && u < p.total_units; u += n_clusters) {
+      Unit U;
+      if (!decode_pair_unit(p, u, U)) continue;
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        if (i == 1 && !U.has_q1) break;
+        if (q_use[i] > 0) {
+          ok = __all_sync(0xffffffffu, pair_wait(&ctl->q_empty[i], (q_use[i] - 1) & 1, ctl,
+                                                 p.timeout_ns, false));
+          if (!ok) break;
+        }
+        stage(U, U.q0 + i * 2 * kTile + static_cast<int>(rank) * kTile);
+        const uint32_t bar = map_to_rank(smem_u32(&ctl->q_full[i]), 0);
+        if (leader && pw == 0 && elect_one()) mbar_arrive_expect_tx(&ctl->q_full[i], 2 * kQBytes);
+        __syncwarp();
+        gathers(&p.tq, bar, sQ + i * kQBytes, 0, 64, 2, kTile * 128, 0);
+        ++q_use[i];
+      }
+      for (int j = 0; ok && j < U.nkv; ++j) {
+        stage(U, j * kTile);
+        const int ns = pair_ns(U, j);
+        const int half = ns >> 1;
+        for (int kv = 0; kv < 2; ++kv) {
+          const int slot = ld % n_slots;
+          const uint32_t use = ld / n_slots;
+          if (use > 0) {
+            ok = __all_sync(0xffffffffu, pair_wait(&ctl->kv_empty[slot], (use - 1) & 1, ctl,
+                                                   p.timeout_ns, false));
+            if (!ok) break;
+          }
+          const uint32_t bar = map_to_rank(smem_u32(&ctl->kv_full[slot]), 0);
+          if (leader && pw == 0 && elect_one())
+            mbar_arrive_expect_tx(&ctl->kv_full[slot], static_cast<uint32_t>(ns) * 256u);
+          __syncwarp();
+          uint8_t* dst = sRing + slot * kPairHalfTileBytes;
+          if (kv == 0)   // K: keys [rank*half, rank*half + half), both column blocks
+            gathers(&p.tk, bar, dst, (static_cast<int>(rank) * half) >> 2, (half >> 2) * 2, 2, 64 * 128, 0);
+          else           // V: keys [0, ns), the column block of this CTA's half of d
+            gathers(&p.tv, bar, dst, 0, ns >> 2, 1, 0, 64 * static_cast<int>(rank));
+          ++ld;
+        }
+      }
+    }
+    // Drain: in the leader, every load of either CTA is counted on these
+    // barriers; the final cluster barrier keeps the peer alive until then.
+    if (leader) {
+      for (int i = 0; i < 2; ++i)
+        if (q_use[i] > 0) mbar_wait_bounded(&ctl->q_full[i], (q_use[i] - 1) & 1, p.timeout_ns);
+      for (uint32_t x = (ld > static_cast<uint32_t>(n_slots) ? ld - n_slots : 0); x < ld; ++x)
+        mbar_wait_bounded(&ctl->kv_full[x % n_slots], (x / n_slots) & 1, p.timeout_ns);
+    }
+  } else if (warp == kPairMmaWarp) {
+    // ================================================================ MMA issuer (leader)
+    if (leader && lane == 0) {
+      const uint32_t q_addr0 = smem_u32(sQ);
+      const uint32_t ring_addr = smem_u32(sRing);
+      const uint32_t idesc_pv = idesc_bf16_f32(256, 128, 0, 1);
+      uint32_t q_use[2] = {0, 0};
+      uint32_t p_use[2] = {0, 0};
+      uint32_t ld = 0;
+      bool ok = true;
+      auto issue_qk = [&](int i, uint32_t k_addr, int ns) {
+        const uint32_t idesc = idesc_bf16_f32(256, ns, 0, 0);
+        const uint32_t q_addr = q_addr0 + i * kQBytes;
+        for (int kk = 0; kk < 8; ++kk) {
+          umma_ss_pair(tmem + (i ? kColS1 : kColS0),
+                       smem_desc_sw128(q_addr + (kk >> 2) * (kTile * 128) + (kk & 3) * 32, 16, 1024),
+                       smem_desc_sw128(k_addr + (kk >> 2) * (64 * 128) + (kk & 3) * 32, 16, 1024),
+                       idesc, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int i, uint32_t v_addr, int ns, bool acc) {
+        const uint32_t tS = tmem + (i ? kColS1 : kColS0);
+        const uint32_t tO = tmem + (i ? kColO1 : kColO0);
+        for (int kk = 0; kk < ns / 16; ++kk)
+          umma_ts_pair(tO, tS + kk * 8, smem_desc_sw128(v_addr + kk * 2048, kTile * 128, 1024),
+                       idesc_pv, (acc || kk > 0) ? 1u : 0u);
+      };
+      for (int u = cluster_id; ok && u < p.total_units; u += n_clusters) {
+        Unit U;
+        if (!decode_pair_unit(p, u, U)) continue;
+        const int nq = U.has_q1 ? 2 : 1;
+#pragma unroll
+        for (int i = 0; i < 2; ++i)
+          if (ok && i < nq) ok = pair_wait(&ctl->q_full[i], q_use[i] & 1, ctl, p.timeout_ns, false);
+        if (!ok) break;
+        int slot_k = ld % n_slots;
+        ok = pair_wait(&ctl->kv_full[slot_k], (ld / n_slots) & 1, ctl, p.timeout_ns, false);
+        if (!ok) break;
+        ++ld;
+        tc_fence_after();
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          if (i >= nq) break;
+          issue_qk(i, ring_addr + slot_k * kPairHalfTileBytes, pair_ns(U, 0));
+          umma_commit_pair(&ctl->s_full[i], 3);
+          if (U.nkv == 1) umma_commit_pair(&ctl->q_empty[i], 3);
+        }
+        umma_commit_pair(&ctl->kv_empty[slot_k], 3);
+        for (int j = 0; j < U.nkv; ++j) {
+          const int slot_v = ld % n_slots;
+          ok = pair_wait(&ctl->kv_full[slot_v], (ld / n_slots) & 1, ctl, p.timeout_ns, false);
+          if (!ok) break;
+          ++ld;
+          const bool more = j + 1 < U.nkv;
+          const int ns = pair_ns(U, j);
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            if (i >= nq) break;
+            ok = pair_wait(&ctl->p_full[i], p_use[i] & 1, ctl, p.timeout_ns, true);
+            if (!ok) break;
+            ++p_use[i];
+            tc_fence_after();
+            issue_pv(i, ring_addr + slot_v * kPairHalfTileBytes, ns, j > 0);
+            if (!more) umma_commit_pair(&ctl->o_final[i], 3);
+            if (i == nq - 1) umma_commit_pair(&ctl->kv_empty[slot_v], 3);
+            if (more) {
+              if (i == 0) {
+                slot_k = ld % n_slots;
+                ok = pair_wait(&ctl->kv_full[slot_k], (ld / n_slots) & 1, ctl, p.timeout_ns, false);
+                if (!ok) break;
+                ++ld;
+                tc_fence_after();
+              }
+              issue_qk(i, ring_addr + slot_k * kPairHalfTileBytes, pair_ns(U, j + 1));
+              umma_commit_pair(&ctl->s_full[i], 3);
+              if (j + 1 == U.nkv - 1) umma_commit_pair(&ctl->q_empty[i], 3);
+              if (i == nq - 1) umma_commit_pair(&ctl->kv_empty[slot_k], 3);
+            }
+          }
+          if (!ok) break;
+        }
+        ++q_use[0];
+        if (nq == 2) ++q_use[1];
+      }
+      umma_commit_pair(&ctl->drained, 1);
+      mbar_wait_bounded(&ctl->drained, 0, p.timeout_ns);
+    }
+    __syncwarp();
+  } else {
+    // ================================================================ softmax (+ correction, epilogue)
+    const int wg = warp >> 2;
+    const int row = threadIdx.x & 127;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + (wg ? kColS1 : kColS0) + lane_off;
+    const uint32_t tO = tmem + (wg ? kColO1 : kColO0) + lane_off;
+    const uint32_t p_full_leader = map_to_rank(smem_u32(&ctl->p_full[wg]), 0);
+    const float sl2 = p.scale_log2;
+    uint32_t s_use = 0, of_use = 0;
+    bool ok = true;
+    for (int u = cluster_id; ok && u < p.total_units; u += n_clusters) {
+      Unit U;
+      if (!decode_pair_unit(p, u, U)) continue;
+      if (wg == 1 && !U.has_q1) continue;
+      float m_run = -INFINITY;
+      float l_run = 0.0f;
+      for (int j = 0; j < U.nkv; ++j) {
+        ok = __all_sync(0xffffffffu, pair_wait(&ctl->s_full[wg], s_use & 1, ctl, p.timeout_ns, false));
+        if (!ok) break;
+        ++s_use;
+        tc_fence_after();
+        const int kvv = kv_valid_of(U, j);
+        const int nchunks = (kvv + 31) >> 5;
+        float x[kTile];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          if (c < nchunks) {
+            uint32_t r[32];
+            tmem_ld32(tS + c * 32, r);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) x[c * 32 + i] = __uint_as_float(r[i]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) x[c * 32 + i] = -INFINITY;
+          }
+        }
+        tmem_wait_ld();
+        if (kvv < kTile) {
+#pragma unroll
+          for (int i = 0; i < kTile; ++i)
+            if (i >= kvv) x[i] = -INFINITY;
+        }
+        float mx = x[0];
+#pragma unroll
+        for (int i = 1; i < kTile; ++i) mx = fmaxf(mx, x[i]);
+        const float m_new = fmaxf(m_run, mx * sl2);
+        const bool need = m_new > m_run + kRescaleThreshold;
+        float alpha = 1.0f;
+        if (need) {
+          alpha = ex2_approx(m_run - m_new);
+          m_run = m_new;
+        }
+        const float neg_m = -m_run;
+        const float rowsum = kvv < kTile ? softmax_to_p<true>(x, nchunks, kvv, sl2, neg_m, tS)
+                                         : softmax_to_p<false>(x, nchunks, kvv, sl2, neg_m, tS);
+        l_run = l_run * alpha + rowsum;
+        if (j > 0 && __any_sync(0xffffffffu, need)) {
+          for (int c = 0; c < 4; ++c) {
+            uint32_t r[32];
+            tmem_ld32(tO + c * 32, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+            tmem_st32(tO + c * 32, r);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(p_full_leader);
+      }
+      if (!ok) break;
+      ok = __all_sync(0xffffffffu, pair_wait(&ctl->o_final[wg], of_use & 1, ctl, p.timeout_ns, false));
+      if (!ok) break;
+      ++of_use;
+      tc_fence_after();
+      const int slot = U.q0 + wg * 2 * kTile + static_cast<int>(rank) * kTile + row;
+      const bool valid = slot < U.n_valid;
+      __nv_bfloat16* dst = nullptr;
+      if (valid) dst = p.out + static_cast<size_t>(pair_row(p, U, slot)) * 128;
+      const float inv_l = 1.0f / l_run;
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tO + c * 32, r);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * inv_l, __uint_as_float(r[2 * i + 1]) * inv_l);
+        if (valid) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            d4[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+        }
+      }
+      tc_fence_before();
+    }
+  }
+
+  tc_fence_before();
+  cluster_sync_all();
+  if (warp == kPairMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, kTmemCols);
   }
 }
 
@@ -479,12 +995,33 @@ static unsigned long long g_timeout_ns = 1000000000ull;
 constexpr int kMaxDevices = 64;
 static int g_dev_state[kMaxDevices];   // 0 unknown, 1 ready, negative error code
 
+static int slots_for(int d) {
+  // K/V ring: as many 128-row tiles as fit next to the two query tiles
+  // within about 200 KB, capped at the ring limit.
+  const int tile = kTile * d * 2;
+  int slots = (200 * 1024 - 2 * tile) / tile;
+  return slots > kMaxSlots ? kMaxSlots : slots;
+}
+
 static size_t smem_bytes_for(int d) {
   const size_t tile = static_cast<size_t>(kTile) * d * 2;
-  size_t bytes = 1024 + tile * (1 + 2 * kStages) + sizeof(SmemCtl);
+  size_t bytes = 1024 + tile * (2 + slots_for(d)) + sizeof(SmemCtl);
   // At most one CTA per SM: each CTA takes all 512 TMEM columns.
   const size_t one_per_sm = 120 * 1024;
   return bytes < one_per_sm ? one_per_sm : bytes;
+}
+
+static int g_sm_count[kMaxDevices];
+static int g_pair_clusters[kMaxDevices];   // co-resident CTA pairs of the pair kernel
+
+static int pair_slots() {
+  int slots = (200 * 1024 - 2 * kTile * 128 * 2) / kPairHalfTileBytes;
+  return slots > kPairMaxSlots ? kPairMaxSlots : slots;
+}
+
+static size_t pair_smem_bytes() {
+  return 1024 + static_cast<size_t>(2 * kTile * 128 * 2) +
+         static_cast<size_t>(pair_slots()) * kPairHalfTileBytes + sizeof(PairCtl);
 }
 
 static int prepare_device(int* dev_out) {
@@ -512,9 +1049,27 @@ static int prepare_device(int* dev_out) {
       return BASA_ERR_CUDA;
     g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
   }
+  size_t smem_max = smem_bytes_for(128) > smem_bytes_for(64) ? smem_bytes_for(128) : smem_bytes_for(64);
   if (cudaFuncSetAttribute(swattn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem_bytes_for(128))) != cudaSuccess)
+                           static_cast<int>(smem_max)) != cudaSuccess)
     return BASA_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&g_sm_count[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      g_sm_count[dev] < 1)
+    return BASA_ERR_CUDA;
+  if (cudaFuncSetAttribute(swattn_fwd_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(pair_smem_bytes())) != cudaSuccess)
+    return BASA_ERR_CUDA;
+  {
+    // How many CTA pairs fit at once (SMs that cannot be paired stay idle).
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * g_sm_count[dev], 1, 1);
+    cfg.blockDim = dim3(kPairThreads, 1, 1);
+    cfg.dynamicSmemBytes = pair_smem_bytes();
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, swattn_fwd_pair_kernel, &cfg) != cudaSuccess || n < 1)
+      return BASA_ERR_CUDA;
+    g_pair_clusters[dev] = n;
+  }
   g_dev_state[dev] = 1;
   return BASA_OK;
 }
@@ -546,6 +1101,7 @@ extern "C" int basa_swattn_fwd(const void* q, const void* k, const void* v, void
   if (!q || !k || !v || !out) return BASA_ERR_INVALID_ARG;
   if (B < 1 || heads < 1) return BASA_ERR_INVALID_ARG;
   if (!std::isfinite(scale)) return BASA_ERR_INVALID_ARG;
+  if (scale < 0.0f) return BASA_ERR_UNSUPPORTED;
   Geometry g;
   int rc = make_geometry(&g, T, H, W, win, shift);
   if (rc) return rc;
@@ -558,13 +1114,38 @@ extern "C" int basa_swattn_fwd(const void* q, const void* k, const void* v, void
   const size_t bytes = static_cast<size_t>(rows) * d * 2;
   if (overlaps(out, q, bytes) || overlaps(out, k, bytes) || overlaps(out, v, bytes))
     return BASA_ERR_ALIAS;
-  const long long q_tiles = (g.nw_max + kTile - 1) / kTile;
-  const long long grid = static_cast<long long>(B) * heads * g.n_windows * q_tiles;
-  if (grid >= (1LL << 31)) return BASA_ERR_UNSUPPORTED;
+  const long long q_pairs = (g.nw_max + 2 * kTile - 1) / (2 * kTile);
+  const long long units = static_cast<long long>(B) * heads * g.n_windows * q_pairs;
+  if (units >= (1LL << 31)) return BASA_ERR_UNSUPPORTED;
 
   int dev = 0;
   rc = prepare_device(&dev);
   if (rc) return rc;
+
+  if (d == 128) {
+    // CTA-pair kernel: units of up to 512 queries, one cluster of two CTAs each.
+    const long long q_quads = (g.nw_max + 4 * kTile - 1) / (4 * kTile);
+    const long long punits = static_cast<long long>(B) * heads * g.n_windows * q_quads;
+    if (punits >= (1LL << 31)) return BASA_ERR_UNSUPPORTED;
+    PairParams pp;
+    memset(&pp, 0, sizeof(pp));
+    if (encode_rows(&pp.tq, q, rows, d) || encode_rows(&pp.tk, k, rows, d) ||
+        encode_rows(&pp.tv, v, rows, d))
+      return BASA_ERR_CUDA;
+    pp.out = static_cast<__nv_bfloat16*>(out);
+    pp.g = g;
+    pp.B = B;
+    pp.heads = heads;
+    pp.q_quads = static_cast<int>(q_quads);
+    pp.total_units = static_cast<int>(punits);
+    pp.n_slots = pair_slots();
+    pp.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+    pp.timeout_ns = g_timeout_ns;
+    const long long clusters = punits < g_pair_clusters[dev] ? punits : g_pair_clusters[dev];
+    swattn_fwd_pair_kernel<<<static_cast<unsigned>(2 * clusters), kPairThreads, pair_smem_bytes(),
+                             static_cast<cudaStream_t>(stream)>>>(pp);
+    return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;
+  }
 
   FwdParams p;
   memset(&p, 0, sizeof(p));
@@ -576,9 +1157,13 @@ extern "C" int basa_swattn_fwd(const void* q, const void* k, const void* v, void
   p.B = B;
   p.heads = heads;
   p.d = d;
-  p.q_tiles = static_cast<int>(q_tiles);
+  p.q_pairs = static_cast<int>(q_pairs);
+  p.total_units = static_cast<int>(units);
+  p.n_slots = slots_for(d);
   p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   p.timeout_ns = g_timeout_ns;
+  // Persistent: one CTA per SM, each walking the units with a stride of the grid.
+  const long long grid = units < g_sm_count[dev] ? units : g_sm_count[dev];
   swattn_fwd_kernel<<<static_cast<unsigned>(grid), kThreads, smem_bytes_for(d),
                       static_cast<cudaStream_t>(stream)>>>(p);
   return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;

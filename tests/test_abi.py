@@ -108,6 +108,7 @@ def test_argument_errors_are_caught_on_the_host(lib):
     assert _fwd(lib, win=(0, 2, 2), out=big) == sw.BASA_ERR_INVALID_ARG
     assert _fwd(lib, scale=float("nan"), out=big) == sw.BASA_ERR_INVALID_ARG
     assert _fwd(lib, scale=float("inf"), out=big) == sw.BASA_ERR_INVALID_ARG
+    assert _fwd(lib, scale=-0.5, out=big) == sw.BASA_ERR_UNSUPPORTED
     assert _fwd(lib, d=96, out=big) == sw.BASA_ERR_UNSUPPORTED
     assert _fwd(lib, d=256, out=big) == sw.BASA_ERR_UNSUPPORTED
     assert _fwd(lib, grid=(1, 1 << 16, 1 << 16), win=(1, 1, 1), out=big) == sw.BASA_ERR_UNSUPPORTED
