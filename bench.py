@@ -44,7 +44,8 @@ HEADLINE = "wan-720p-21x45x80-w7x15x16"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_NAME = "swattn_fwd_kernel"
 KERNEL_SOURCES = ["shifted_window_attention_swattn_b200/csrc/swattn_sm100.cu",
-                  "shifted_window_attention_swattn_b200/csrc/ptx_sm100.cuh"]
+                  "shifted_window_attention_swattn_b200/csrc/ptx_sm100.cuh",
+                  "shifted_window_attention_swattn_b200/csrc/softmax_sm100.cuh"]
 
 
 def kernel_source_hash() -> str:

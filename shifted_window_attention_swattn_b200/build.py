@@ -13,6 +13,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 SOURCES = [os.path.join(HERE, "csrc", "swattn_sm100.cu")]
 DEPS = SOURCES + [os.path.join(HERE, "csrc", "ptx_sm100.cuh"),
+                  os.path.join(HERE, "csrc", "softmax_sm100.cuh"),
                   os.path.join(ROOT, "include", "basa_swattn.h")]
 LIB = os.path.join(HERE, "libbasa_swattn.so")
 

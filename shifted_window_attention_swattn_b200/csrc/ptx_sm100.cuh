@@ -107,10 +107,11 @@ __device__ __forceinline__ uint32_t map_to_rank(uint32_t smem_addr, uint32_t ran
 }
 
 // Arrive on an mbarrier given by its shared::cluster address (possibly in the
-// peer CTA), with release semantics at cluster scope.
+// peer CTA).  Default (CTA-scope release) semantics: what this orders is
+// tensor-memory work, which the tcgen05 fences around the arrive and the
+// matching wait already order.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-               : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {

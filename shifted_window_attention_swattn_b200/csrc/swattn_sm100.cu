@@ -38,11 +38,13 @@
 #include <cmath>
 #include <math.h>
 #include <mutex>
+#include <type_traits>
 #include <stdint.h>
 #include <string.h>
 
 #include "basa_swattn.h"
 #include "ptx_sm100.cuh"
+#include "softmax_sm100.cuh"
 
 namespace swattn {
 
@@ -226,36 +228,6 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint3
   for (int kk = 0; kk < ksteps; ++kk)
     umma_ts(tmem_o, tmem_p + kk * 8, smem_desc_sw128(v_addr + kk * 2048, kTile * 128, 1024), idesc,
             (accumulate || kk > 0) ? 1u : 0u);
-}
-
-// P = exp2(x * scale_log2 - m) for one S row held in registers, packed to
-// bf16 pairs and stored over the front of the S row in TMEM; returns the row
-// sum of the fp32 values.  kPartial: columns >= kv_valid are padding keys and
-// get P = 0.
-template <bool kPartial>
-__device__ __forceinline__ float softmax_to_p(const float (&x)[kTile], int nchunks, int kv_valid,
-                                              float sl2, float neg_m, uint32_t tS) {
-  float rowsum = 0.0f;
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    if (c < nchunks) {
-      uint32_t pk[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int col = c * 32 + 2 * i;
-        float p0 = ex2_approx(fmaf(x[col], sl2, neg_m));
-        float p1 = ex2_approx(fmaf(x[col + 1], sl2, neg_m));
-        if (kPartial) {
-          p0 = col < kv_valid ? p0 : 0.0f;
-          p1 = col + 1 < kv_valid ? p1 : 0.0f;
-        }
-        rowsum += p0 + p1;
-        pk[i] = pack_bf16x2(p0, p1);
-      }
-      tmem_st16(tS + c * 16, pk);   // P overwrites the front of the S row
-    }
-  }
-  return rowsum;
 }
 
 __global__ void __launch_bounds__(kThreads, 1) swattn_fwd_kernel(const __grid_constant__ FwdParams p) {
@@ -489,9 +461,7 @@ __global__ void __launch_bounds__(kThreads, 1) swattn_fwd_kernel(const __grid_co
           for (int i = 0; i < kTile; ++i)
             if (i >= kvv) x[i] = -INFINITY;
         }
-        float mx = x[0];
-#pragma unroll
-        for (int i = 1; i < kTile; ++i) mx = fmaxf(mx, x[i]);
+        const float mx = row_max128(x);
         const float m_new = fmaxf(m_run, mx * sl2);
         const bool need = m_new > m_run + kRescaleThreshold;
         float alpha = 1.0f;
@@ -500,8 +470,8 @@ __global__ void __launch_bounds__(kThreads, 1) swattn_fwd_kernel(const __grid_co
           m_run = m_new;
         }
         const float neg_m = -m_run;
-        const float rowsum = kvv < kTile ? softmax_to_p<true>(x, nchunks, kvv, sl2, neg_m, tS)
-                                         : softmax_to_p<false>(x, nchunks, kvv, sl2, neg_m, tS);
+        const float rowsum = kvv < kTile ? softmax_tile_to_p<true>(x, nchunks, kvv, sl2, neg_m, tS)
+                                         : softmax_tile_to_p<false>(x, nchunks, kvv, sl2, neg_m, tS);
         l_run = l_run * alpha + rowsum;
         if (j > 0 && __any_sync(0xffffffffu, need)) {
           // O_i holds P V of tiles 0..j-1 (complete: S_i(j) was issued after
@@ -836,7 +806,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
 #pragma unroll
           for (int i = 0; i < 2; ++i) {
             if (i >= nq) break;
-            ok = pair_wait(&ctl->p_full[i], p_use[i] & 1, ctl, p.timeout_ns, true);
+            ok = pair_wait(&ctl->p_full[i], p_use[i] & 1, ctl, p.timeout_ns, false);
             if (!ok) break;
             ++p_use[i];
             tc_fence_after();
@@ -909,9 +879,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           for (int i = 0; i < kTile; ++i)
             if (i >= kvv) x[i] = -INFINITY;
         }
-        float mx = x[0];
-#pragma unroll
-        for (int i = 1; i < kTile; ++i) mx = fmaxf(mx, x[i]);
+        const float mx = row_max128(x);
         const float m_new = fmaxf(m_run, mx * sl2);
         const bool need = m_new > m_run + kRescaleThreshold;
         float alpha = 1.0f;
@@ -920,8 +888,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           m_run = m_new;
         }
         const float neg_m = -m_run;
-        const float rowsum = kvv < kTile ? softmax_to_p<true>(x, nchunks, kvv, sl2, neg_m, tS)
-                                         : softmax_to_p<false>(x, nchunks, kvv, sl2, neg_m, tS);
+        const float rowsum = kvv < kTile ? softmax_tile_to_p<true>(x, nchunks, kvv, sl2, neg_m, tS)
+                                         : softmax_tile_to_p<false>(x, nchunks, kvv, sl2, neg_m, tS);
         l_run = l_run * alpha + rowsum;
         if (j > 0 && __any_sync(0xffffffffu, need)) {
           for (int c = 0; c < 4; ++c) {
