@@ -42,7 +42,7 @@ sys.path.insert(0, ROOT)
 METRIC = "shifted-window attn fwd TFLOP/s & % of B200 BF16 peak; speedup vs full attn"
 HEADLINE = "wan-720p-21x45x80-w7x15x16"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_NAME = "swattn_fwd_kernel"
+KERNEL_NAME = "swattn_fwd_pair_kernel"   # the head-dim-128 kernel the headline workload runs
 KERNEL_SOURCES = ["shifted_window_attention_swattn_b200/csrc/swattn_sm100.cu",
                   "shifted_window_attention_swattn_b200/csrc/ptx_sm100.cuh",
                   "shifted_window_attention_swattn_b200/csrc/softmax_sm100.cuh"]
@@ -68,16 +68,24 @@ def load_peaks():
 
 def load_traffic():
     """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current kernel source."""
-    path = os.path.join(ROOT, "profiles", "swattn_fwd_kernel_traffic.json")
+    on the current kernel sources (key = value lines, '#' comments)."""
+    path = os.path.join(ROOT, "profiles", "swattn_fwd_pair_kernel_wan720p_traffic.txt")
+    rec = {}
     try:
         with open(path) as f:
-            rec = json.load(f)
-    except (OSError, ValueError):
+            for line in f:
+                line = line.strip()
+                if line and not line.startswith("#") and "=" in line:
+                    k, v = (x.strip() for x in line.split("=", 1))
+                    rec[k] = v
+    except OSError:
         return None
     if rec.get("kernel_source_hash") != kernel_source_hash():
         return None
-    return rec
+    try:
+        return {"dram_bytes_per_launch": float(rec["dram_bytes_per_launch"])}
+    except (KeyError, ValueError):
+        return None
 
 
 # ---------------------------------------------------------------- clocks
