@@ -216,6 +216,22 @@ def wl_config(wl, extra=None):
     return cfg
 
 
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """Maximum of a per-rank float over all ranks (identity on one rank)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(flops_per_rank: float, world: int, ms_max: float) -> float:
+    """Throughput of the whole job: every rank's FLOPs over the slowest rank's time."""
+    return flops_per_rank * world / (ms_max / 1e3) / 1e12
+
+
 def dist_env():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -379,13 +395,9 @@ def run_native(args):
     if sw.last_device_error() != sw.BASA_OK:
         raise RuntimeError("device-side wait timed out in the timed region")
     launches = args.steps * len(wl.shifts)
-    t_max = ms_total
-    if world > 1:
-        t = torch.tensor([ms_total], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        t_max = float(t.item())
+    t_max = max_over_ranks(ms_total, world, device)
     ms_per_step = t_max / args.steps
-    value = f_step * args.steps * world / (t_max / 1e3) / 1e12
+    value = whole_job_tflops(f_step * args.steps, world, t_max)
     ms_launch = ms_total / launches
     achieved = f_layer / (ms_launch / 1e3) / 1e12
 
@@ -419,12 +431,8 @@ def run_native(args):
         b.record(stream)
         torch.cuda.synchronize()
         barrier()
-        e2e_ms = a.elapsed_time(b)
-        if world > 1:
-            t = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = {"value": f_step * e2e_steps * world / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+        e2e_ms = max_over_ranks(a.elapsed_time(b), world, device)
+        e2e = {"value": whole_job_tflops(f_step * e2e_steps, world, e2e_ms), "unit": "TFLOP/s",
                "h2d_bytes_per_step": 3 * q.numel() * 2,
                "d2h_bytes_per_step": len(wl.shifts) * q.numel() * 2,
                "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps,

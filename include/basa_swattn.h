@@ -106,6 +106,14 @@ int basa_swattn_last_device_error(void* stream);
  */
 int basa_swattn_set_wait_timeout_ns(unsigned long long ns);
 
+/*
+ * Test hook for the bounded-wait error path (not part of the method): while
+ * `on` is non-zero, every launch's MMA issuer first waits on a barrier that
+ * nothing arrives on, so the launch times out after the wait limit, stops,
+ * drains and reports BASA_ERR_DEVICE.  Off by default.
+ */
+int basa_swattn_set_test_stall(int on);
+
 /* Static, human-readable text for a BASA_* code. */
 const char* basa_strerror(int code);
 

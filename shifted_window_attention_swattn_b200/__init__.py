@@ -69,6 +69,8 @@ def _load():
         lib.basa_swattn_last_device_error.restype = ci
         lib.basa_swattn_set_wait_timeout_ns.argtypes = [ctypes.c_ulonglong]
         lib.basa_swattn_set_wait_timeout_ns.restype = ci
+        lib.basa_swattn_set_test_stall.argtypes = [ci]
+        lib.basa_swattn_set_test_stall.restype = ci
         lib.basa_strerror.argtypes = [ci]
         lib.basa_strerror.restype = ctypes.c_char_p
         _lib = lib
@@ -213,3 +215,8 @@ def last_device_error(stream=None) -> int:
 
 def set_wait_timeout_ns(ns: int) -> None:
     _load().basa_swattn_set_wait_timeout_ns(int(ns))
+
+
+def set_test_stall(on: bool) -> None:
+    """Test hook: make every launch's MMA issuer wait on a barrier nothing arrives on."""
+    _load().basa_swattn_set_test_stall(1 if on else 0)

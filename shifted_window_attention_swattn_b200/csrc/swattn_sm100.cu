@@ -36,6 +36,7 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
+#include <cstddef>
 #include <math.h>
 #include <mutex>
 #include <type_traits>
@@ -143,6 +144,7 @@ struct __align__(64) FwdParams {
   int n_slots;                  // K/V ring depth (tiles)
   float scale_log2;             // scale * log2(e)
   unsigned long long timeout_ns;
+  int stall;                    // test hook: the MMA issuer first waits on a barrier nothing arrives on
 };
 
 struct SmemCtl {
@@ -154,12 +156,26 @@ struct SmemCtl {
   uint64_t p_full[2];           // P_i is in TMEM and O_i is rescaled
   uint64_t o_final[2];          // last P V of the unit for tile i is done
   uint64_t drained;             // every MMA of the CTA is done
+  uint64_t never;               // test hook: never arrived on
   uint32_t tmem_base;
   int abort;
-  int rows[kProducers][kTile / kProducers];   // gather coordinates staged per producer warp
+  // gather coordinates staged per producer warp, read back 4 at a time as int4
+  alignas(16) int rows[kProducers][kTile / kProducers];
 };
 
+static_assert(offsetof(SmemCtl, rows) % 16 == 0, "int4 reads of staged rows");
+static_assert(offsetof(SmemCtl, q_full) % 8 == 0, "mbarriers are 8-byte aligned");
+
 __device__ int g_device_error = 0;
+
+// Waits that drain work already in flight (MMAs, TMA loads) before TMEM is
+// released or the CTA exits get at least this long, whatever the caller's
+// wait limit: in-flight hardware work always finishes, and cutting these
+// waits short would release resources it still uses.
+constexpr unsigned long long kDrainMinNs = 200ull * 1000 * 1000;
+__device__ __forceinline__ unsigned long long drain_ns(unsigned long long t) {
+  return t > kDrainMinNs ? t : kDrainMinNs;
+}
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, SmemCtl* ctl,
                                               unsigned long long timeout_ns) {
@@ -257,6 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1) swattn_fwd_kernel(const __grid_co
       mbar_init(&ctl->kv_empty[s], 1);
     }
     mbar_init(&ctl->drained, 1);
+    mbar_init(&ctl->never, 1);
     ctl->abort = 0;
     fence_barrier_init();
   }
@@ -338,9 +355,9 @@ __global__ void __launch_bounds__(kThreads, 1) swattn_fwd_kernel(const __grid_co
     // Drain: every load issued has landed before the CTA can exit.  In the
     // normal flow these phases completed long ago and the waits return at once.
     for (int i = 0; i < 2; ++i)
-      if (q_use[i] > 0) mbar_wait_bounded(&ctl->q_full[i], (q_use[i] - 1) & 1, p.timeout_ns);
+      if (q_use[i] > 0) mbar_wait_bounded(&ctl->q_full[i], (q_use[i] - 1) & 1, drain_ns(p.timeout_ns));
     for (uint32_t x = (ld > static_cast<uint32_t>(n_slots) ? ld - n_slots : 0); x < ld; ++x)
-      mbar_wait_bounded(&ctl->kv_full[x % n_slots], (x / n_slots) & 1, p.timeout_ns);
+      mbar_wait_bounded(&ctl->kv_full[x % n_slots], (x / n_slots) & 1, drain_ns(p.timeout_ns));
   } else if (warp == kMmaWarp) {
     // ================================================================ MMA issuer
     if (lane == 0) {
@@ -351,7 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1) swattn_fwd_kernel(const __grid_co
       uint32_t q_use[2] = {0, 0};
       uint32_t p_use[2] = {0, 0};
       uint32_t ld = 0;        // ring tiles consumed
-      bool ok = true;
+      bool ok = !p.stall || wait_or_abort(&ctl->never, 0, ctl, p.timeout_ns);
       for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
         Unit U;
         if (!decode_unit(p, u, U)) continue;
@@ -416,7 +433,7 @@ __global__ void __launch_bounds__(kThreads, 1) swattn_fwd_kernel(const __grid_co
       }
       // Drain every MMA this thread issued before TMEM is released.
       umma_commit(&ctl->drained);
-      mbar_wait_bounded(&ctl->drained, 0, p.timeout_ns);
+      mbar_wait_bounded(&ctl->drained, 0, drain_ns(p.timeout_ns));
     }
     __syncwarp();
   } else {
@@ -561,6 +578,7 @@ struct __align__(64) PairParams {
   int n_slots;
   float scale_log2;
   unsigned long long timeout_ns;
+  int stall;                    // test hook: the MMA issuer first waits on a barrier nothing arrives on
 };
 
 struct PairCtl {
@@ -572,10 +590,15 @@ struct PairCtl {
   uint64_t p_full[2];           // leader: P_i written (and O_i rescaled) in both CTAs
   uint64_t o_final[2];          // both: last P V of the unit for tile i done
   uint64_t drained;             // leader: every MMA done
+  uint64_t never;               // test hook: never arrived on
   uint32_t tmem_base;
   int abort;
-  int rows[kPairProducers][kTile];   // gather coordinates staged per producer warp
+  // gather coordinates staged per producer warp, read back 4 at a time as int4
+  alignas(16) int rows[kPairProducers][kTile];
 };
+
+static_assert(offsetof(PairCtl, rows) % 16 == 0, "int4 reads of staged rows");
+static_assert(offsetof(PairCtl, q_full) % 8 == 0, "mbarriers are 8-byte aligned");
 
 __device__ __forceinline__ bool pair_wait(uint64_t* bar, uint32_t parity, PairCtl* ctl,
                                           unsigned long long timeout_ns, bool cluster_scope) {
@@ -648,6 +671,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       mbar_init(&ctl->kv_empty[s], 1);
     }
     mbar_init(&ctl->drained, 1);
+    mbar_init(&ctl->never, 1);
     ctl->abort = 0;
     fence_barrier_init();
   }
@@ -744,9 +768,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     // barriers; the final cluster barrier keeps the peer alive until then.
     if (leader) {
       for (int i = 0; i < 2; ++i)
-        if (q_use[i] > 0) mbar_wait_bounded(&ctl->q_full[i], (q_use[i] - 1) & 1, p.timeout_ns);
+        if (q_use[i] > 0) mbar_wait_bounded(&ctl->q_full[i], (q_use[i] - 1) & 1, drain_ns(p.timeout_ns));
       for (uint32_t x = (ld > static_cast<uint32_t>(n_slots) ? ld - n_slots : 0); x < ld; ++x)
-        mbar_wait_bounded(&ctl->kv_full[x % n_slots], (x / n_slots) & 1, p.timeout_ns);
+        mbar_wait_bounded(&ctl->kv_full[x % n_slots], (x / n_slots) & 1, drain_ns(p.timeout_ns));
     }
   } else if (warp == kPairMmaWarp) {
     // ================================================================ MMA issuer (leader)
@@ -757,7 +781,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       uint32_t q_use[2] = {0, 0};
       uint32_t p_use[2] = {0, 0};
       uint32_t ld = 0;
-      bool ok = true;
+      bool ok = !p.stall || pair_wait(&ctl->never, 0, ctl, p.timeout_ns, false);
       auto issue_qk = [&](int i, uint32_t k_addr, int ns) {
         const uint32_t idesc = idesc_bf16_f32(256, ns, 0, 0);
         const uint32_t q_addr = q_addr0 + i * kQBytes;
@@ -833,7 +857,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         if (nq == 2) ++q_use[1];
       }
       umma_commit_pair(&ctl->drained, 1);
-      mbar_wait_bounded(&ctl->drained, 0, p.timeout_ns);
+      mbar_wait_bounded(&ctl->drained, 0, drain_ns(p.timeout_ns));
     }
     __syncwarp();
   } else {
@@ -960,6 +984,7 @@ __global__ void index_map_kernel(Geometry g, int32_t* tos) {
 static std::mutex g_mutex;
 static PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 static unsigned long long g_timeout_ns = 1000000000ull;
+static int g_stall = 0;   // test hook, see basa_swattn_set_test_stall
 constexpr int kMaxDevices = 64;
 static int g_dev_state[kMaxDevices];   // 0 unknown, 1 ready, negative error code
 
@@ -1109,6 +1134,7 @@ extern "C" int basa_swattn_fwd(const void* q, const void* k, const void* v, void
     pp.n_slots = pair_slots();
     pp.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
     pp.timeout_ns = g_timeout_ns;
+    pp.stall = g_stall;
     const long long clusters = punits < g_pair_clusters[dev] ? punits : g_pair_clusters[dev];
     swattn_fwd_pair_kernel<<<static_cast<unsigned>(2 * clusters), kPairThreads, pair_smem_bytes(),
                              static_cast<cudaStream_t>(stream)>>>(pp);
@@ -1130,6 +1156,7 @@ extern "C" int basa_swattn_fwd(const void* q, const void* k, const void* v, void
   p.n_slots = slots_for(d);
   p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   p.timeout_ns = g_timeout_ns;
+  p.stall = g_stall;
   // Persistent: one CTA per SM, each walking the units with a stride of the grid.
   const long long grid = units < g_sm_count[dev] ? units : g_sm_count[dev];
   swattn_fwd_kernel<<<static_cast<unsigned>(grid), kThreads, smem_bytes_for(d),
@@ -1205,6 +1232,12 @@ extern "C" int basa_swattn_last_device_error(void* stream) {
 extern "C" int basa_swattn_set_wait_timeout_ns(unsigned long long ns) {
   std::lock_guard<std::mutex> lock(g_mutex);
   g_timeout_ns = ns;
+  return BASA_OK;
+}
+
+extern "C" int basa_swattn_set_test_stall(int on) {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  g_stall = on ? 1 : 0;
   return BASA_OK;
 }
 
