@@ -8,9 +8,10 @@
 // dense attention backend; here they never touch memory:
 //
 //   * the roll + partition is the row list of TMA tile::gather4 loads (each
-//     load brings 4 arbitrary token rows of Q, K or V into a 128-byte-swizzled
-//     shared-memory tile), so windows are gathered straight from the
-//     [B, T*H*W, heads, d] tensors;
+//     load brings 4 arbitrary token rows x 64 columns of Q, K or V into a
+//     128-byte-swizzled shared-memory tile), so windows are gathered straight
+//     from the [B, T*H*W, heads, d] tensors.  Each producer lane computes the
+//     rows of its own gathers and a warp issues all of them in one instruction;
 //   * S = Q K^T and O += P V run on tcgen05 tensor cores with S, P and O in
 //     tensor memory (TMEM);
 //   * softmax is online (running max / sum per query row, one thread per row),
@@ -19,11 +20,15 @@
 //   * the inverse roll is the row address of the output store: each query's
 //     result is written back to the token row it was gathered from.
 //
-// One CTA handles one 128-query tile of one window of one (batch, head):
-//   warps 0-3  softmax, O correction and epilogue (thread t owns query row t)
-//   warp  4    TMA producer (Q once, then K/V tiles through a 2-stage ring)
-//   warp  5    TMEM owner and MMA issuer (one elected lane)
-// TMEM columns: S0 [0,128) S1 [128,256) O [256,256+d) P0 [384,448) P1 [448,512).
+// Two persistent kernels share this pipeline.  A work unit is a run of query
+// tiles of one window of one (batch, head); each unit streams the window's
+// K/V tiles through a shared-memory ring, and two query tiles per CTA are
+// processed in ping-pong (softmax of one tile overlaps the MMAs of the other).
+//   * swattn_fwd_pair_kernel (d = 128): clusters of two CTAs issue M = 256
+//     MMAs with cta_group::2; each SM loads half of every K/V tile;
+//   * swattn_fwd_kernel (any supported d, one CTA per SM): M = 128 MMAs.
+// TMEM columns: S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512); P_i is
+// bf16 over the front of S_i.
 //
 // Every mbarrier wait is bounded by a host-set timeout; a wait that runs out
 // raises a shared abort flag and a library-wide error word, every role stops
@@ -159,11 +164,8 @@ struct SmemCtl {
   uint64_t never;               // test hook: never arrived on
   uint32_t tmem_base;
   int abort;
-  // gather coordinates staged per producer warp, read back 4 at a time as int4
-  alignas(16) int rows[kProducers][kTile / kProducers];
 };
 
-static_assert(offsetof(SmemCtl, rows) % 16 == 0, "int4 reads of staged rows");
 static_assert(offsetof(SmemCtl, q_full) % 8 == 0, "mbarriers are 8-byte aligned");
 
 __device__ int g_device_error = 0;
@@ -223,6 +225,41 @@ __device__ __forceinline__ int unit_row(const FwdParams& p, const Unit& U, int s
 __device__ __forceinline__ int kv_valid_of(const Unit& U, int j) {
   const int left = U.n_valid - j * kTile;
   return left < kTile ? left : kTile;
+}
+
+// Rows of slots s .. s+3 of unit U in the 2D [B*N*heads, d] view of Q/K/V/out,
+// row = (b*N + token)*heads + h; slots at or past n_valid repeat the last valid
+// slot's row.  The same tokens as slot_token(), slot by slot: the first slot is
+// split into (s_t, s_h, s_w) with divisions, the next three step along the
+// raster order.
+__device__ __forceinline__ void unit_rows4(const Geometry& g, const Unit& U, int heads, int s,
+                                           int r[4]) {
+  int sw = s % U.e[2];
+  const int q = s / U.e[2];
+  int sh = q % U.e[1];
+  int st = q / U.e[1];
+  const int base_t = U.m[0] * g.w[0] + g.delta[0];
+  const int base_h = U.m[1] * g.w[1] + g.delta[1];
+  const int base_w = U.m[2] * g.w[2] + g.delta[2];
+  const int tok0 = U.b * g.N;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const bool pad = st >= U.e[0];
+    int pt = base_t + (pad ? U.e[0] - 1 : st);
+    int ph = base_h + (pad ? U.e[1] - 1 : sh);
+    int pw = base_w + (pad ? U.e[2] - 1 : sw);
+    if (pt >= g.n[0]) pt -= g.n[0];
+    if (ph >= g.n[1]) ph -= g.n[1];
+    if (pw >= g.n[2]) pw -= g.n[2];
+    r[k] = (tok0 + (pt * g.n[1] + ph) * g.n[2] + pw) * heads + U.h;
+    if (++sw == U.e[2]) {
+      sw = 0;
+      if (++sh == U.e[1]) {
+        sh = 0;
+        ++st;
+      }
+    }
+  }
 }
 
 // S_i (+)= Q_i K^T over the head dimension: d/16 MMAs of M=128, N=n_s, K=16.
@@ -293,34 +330,26 @@ __global__ void __launch_bounds__(kThreads, 1) swattn_fwd_kernel(const __grid_co
 
   if (warp >= kProducerWarp0 && warp < kProducerWarp0 + kProducers) {
     // ================================================================ TMA producers
-    // Each producer warp loads rows [pw*64, pw*64+64) of every tile.  All lanes
-    // compute gather coordinates into shared memory; the warp then walks them
-    // with warp-uniform control flow and one elected lane issues each load.
+    // A tile is 32 * ncb gathers (4 rows x 64 columns each); gather n covers
+    // rows 4 (n / ncb) + [0, 4) and column block n % ncb and belongs to lane
+    // n / 2 of producer warp n % 2, which computes its own row coordinates.
+    // Every lane with a gather issues it in the same instruction.
     const int pw = warp - kProducerWarp0;
-    constexpr int kRowsPer = kTile / kProducers;
     const int ncb = d / 64;   // 128-byte column blocks per row
     const uint32_t half_bytes = tile_bytes / kProducers;
-    int* rows = ctl->rows[pw];
-    const int4* rows4 = reinterpret_cast<const int4*>(rows);
     uint32_t q_use[2] = {0, 0};
     uint32_t ld = 0;          // loads issued into the ring
     bool ok = true;
-    auto stage_rows = [&](const Unit& U, int slot0) {
-      __syncwarp();
-      for (int x = lane; x < kRowsPer; x += 32) rows[x] = unit_row(p, U, slot0 + pw * kRowsPer + x);
-      __syncwarp();
-    };
-    auto issue = [&](const CUtensorMap* map, uint64_t* bar, uint8_t* tile) {
+    auto issue = [&](const Unit& U, int slot0, const CUtensorMap* map, uint64_t* bar, uint8_t* tile) {
       if (elect_one()) mbar_arrive_expect_tx(bar, half_bytes);
       __syncwarp();
-      uint8_t* dst = tile + pw * kRowsPer * 128;
-      for (int g = 0; g < kRowsPer / 4; ++g) {
-        const int4 r = rows4[g];
-        if (elect_one())
-          for (int c = 0; c < ncb; ++c)
-            tma_gather4(map, bar, dst + c * (kTile * 128) + g * 512, c * 64, r.x, r.y, r.z, r.w);
-        __syncwarp();
+      for (int n = pw + kProducers * lane; n < 32 * ncb; n += 32 * kProducers) {
+        const int grp = n / ncb, c = n - grp * ncb;
+        int r[4];
+        unit_rows4(p.g, U, p.heads, slot0 + 4 * grp, r);
+        tma_gather4(map, bar, tile + c * (kTile * 128) + grp * 512, c * 64, r[0], r[1], r[2], r[3]);
       }
+      __syncwarp();
     };
     for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
       Unit U;
@@ -333,12 +362,10 @@ __global__ void __launch_bounds__(kThreads, 1) swattn_fwd_kernel(const __grid_co
                           wait_or_abort(&ctl->q_empty[i], (q_use[i] - 1) & 1, ctl, p.timeout_ns));
           if (!ok) break;
         }
-        stage_rows(U, U.q0 + i * kTile);
-        issue(&p.tq, &ctl->q_full[i], sQ + i * tile_bytes);
+        issue(U, U.q0 + i * kTile, &p.tq, &ctl->q_full[i], sQ + i * tile_bytes);
         ++q_use[i];
       }
       for (int j = 0; ok && j < U.nkv; ++j) {
-        stage_rows(U, j * kTile);
         for (int kv = 0; kv < 2; ++kv) {
           const int slot = ld % n_slots;
           const uint32_t use = ld / n_slots;
@@ -347,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1) swattn_fwd_kernel(const __grid_co
                             wait_or_abort(&ctl->kv_empty[slot], (use - 1) & 1, ctl, p.timeout_ns));
             if (!ok) break;
           }
-          issue(kv == 0 ? &p.tk : &p.tv, &ctl->kv_full[slot], sRing + slot * tile_bytes);
+          issue(U, j * kTile, kv == 0 ? &p.tk : &p.tv, &ctl->kv_full[slot], sRing + slot * tile_bytes);
           ++ld;
         }
       }
@@ -554,17 +581,20 @@ __global__ void __launch_bounds__(kThreads, 1) swattn_fwd_kernel(const __grid_co
 // head dimension of V), so each SM loads half the K/V bytes of the one-CTA
 // kernel and each MMA reads half of its B operand from each SM.
 //
-// Per CTA: warps 0-7 softmax (two query tiles, ping-pong), warps 8-10 TMA
-// producers, warp 11 TMEM owner; in the leader CTA (rank 0) warp 11 also
-// issues every MMA of the pair.  Barriers that gate MMAs (q_full, kv_full,
+// Per CTA: warps 0-7 softmax (two query tiles, ping-pong), then the TMA
+// producer warps, then the TMEM owner warp, which in the leader CTA (rank 0)
+// also issues every MMA of the pair.  Barriers that gate MMAs (q_full, kv_full,
 // p_full) live in the leader and count both CTAs; barriers that MMAs signal
 // (s_full, o_final, q_empty, kv_empty) are arrived on in both CTAs.
 // ============================================================================
 
-constexpr int kPairThreads = 384;   // 12 warps
+#ifndef SWATTN_PAIR_PRODUCERS
+#define SWATTN_PAIR_PRODUCERS 3
+#endif
 constexpr int kPairProducer0 = 8;
-constexpr int kPairProducers = 3;
-constexpr int kPairMmaWarp = 11;
+constexpr int kPairProducers = SWATTN_PAIR_PRODUCERS;
+constexpr int kPairMmaWarp = kPairProducer0 + kPairProducers;
+constexpr int kPairThreads = (kPairMmaWarp + 1) * 32;
 constexpr int kPairHalfTileBytes = 16384;   // a K half (64 keys x 128) or V half (128 keys x 64)
 constexpr int kPairMaxSlots = 12;
 
@@ -593,11 +623,8 @@ struct PairCtl {
   uint64_t never;               // test hook: never arrived on
   uint32_t tmem_base;
   int abort;
-  // gather coordinates staged per producer warp, read back 4 at a time as int4
-  alignas(16) int rows[kPairProducers][kTile];
 };
 
-static_assert(offsetof(PairCtl, rows) % 16 == 0, "int4 reads of staged rows");
 static_assert(offsetof(PairCtl, q_full) % 8 == 0, "mbarriers are 8-byte aligned");
 
 __device__ __forceinline__ bool pair_wait(uint64_t* bar, uint32_t parity, PairCtl* ctl,
@@ -691,35 +718,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
 
   if (warp >= kPairProducer0 && warp < kPairProducer0 + kPairProducers) {
     // ================================================================ TMA producers
-    // Gathers of every tile are spread over the three producer warps; each
-    // warp stages the tile's 128 row coordinates in shared memory, walks them
-    // with warp-uniform control flow, and one elected lane issues each load.
-    // Loads land in this CTA and are counted on the leader's barriers.
+    // Gathers of every tile are spread over the producer warps' lanes (see
+    // `gathers`).  Loads land in this CTA and are counted on the leader's barriers.
     const int pw = warp - kPairProducer0;
-    int* rows = ctl->rows[pw];
-    const int4* rows4 = reinterpret_cast<const int4*>(rows);
     uint32_t q_use[2] = {0, 0};
     uint32_t ld = 0;
     bool ok = true;
-    auto stage = [&](const Unit& U, int slot0) {
-      __syncwarp();
-#pragma unroll
-      for (int x = 0; x < 4; ++x) rows[lane * 4 + x] = pair_row(p, U, slot0 + lane * 4 + x);
-      __syncwarp();
-    };
-    // `count` gathers numbered 0..count-1; gather n covers row group
-    // first_group + n / nblk and column block n % nblk, at dst + (n / nblk) * 512
-    // + (n % nblk) * blk_stride, column col0 + 64 * (n % nblk).
-    auto gathers = [&](const CUtensorMap* map, uint32_t bar_leader, uint8_t* dst, int first_group,
-                       int count, int nblk, int blk_stride, int col0) {
-      for (int n = pw; n < count; n += kPairProducers) {
-        const int grp = n / nblk, blk = n - grp * nblk;
-        const int4 r = rows4[first_group + grp];
-        if (elect_one())
-          tma_gather4_pair(map, bar_leader, dst + grp * 512 + blk * blk_stride, col0 + 64 * blk, r.x,
-                           r.y, r.z, r.w);
-        __syncwarp();
+    // `count` gathers numbered 0..count-1 cover slots slot0 + [0, 4 * count / nblk):
+    // gather n covers row group n / nblk (slots slot0 + 4 (n / nblk) + [0, 4)) and
+    // column block n % nblk, landing at dst + (n / nblk) * 512 + (n % nblk) * blk_stride,
+    // columns col0 + 64 * (n % nblk).  Gather n belongs to lane (n / P) mod 32 of
+    // producer warp n mod P (P producer warps), which computes its own four row
+    // coordinates; every lane with a gather issues it in the same instruction, so
+    // a warp puts up to 32 gathers in flight per issue.
+    auto gathers = [&](const Unit& U, const CUtensorMap* map, uint32_t bar_leader, uint8_t* dst,
+                       int slot0, int count, int nblk, int blk_stride, int col0) {
+      for (int base = 0; base < count; base += 32 * kPairProducers) {
+        const int n = base + pw + kPairProducers * lane;
+        if (n < count) {
+          const int grp = n / nblk, blk = n - grp * nblk;
+          int r[4];
+          unit_rows4(p.g, U, p.heads, slot0 + 4 * grp, r);
+          tma_gather4_pair(map, bar_leader, dst + grp * 512 + blk * blk_stride, col0 + 64 * blk, r[0],
+                           r[1], r[2], r[3]);
+        }
       }
+      __syncwarp();
     };
     for (int u = cluster_id; ok && u < p.total_units; u += n_clusters) {
       Unit U;
@@ -732,15 +756,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                                                  p.timeout_ns, false));
           if (!ok) break;
         }
-        stage(U, U.q0 + i * 2 * kTile + static_cast<int>(rank) * kTile);
         const uint32_t bar = map_to_rank(smem_u32(&ctl->q_full[i]), 0);
         if (leader && pw == 0 && elect_one()) mbar_arrive_expect_tx(&ctl->q_full[i], 2 * kQBytes);
         __syncwarp();
-        gathers(&p.tq, bar, sQ + i * kQBytes, 0, 64, 2, kTile * 128, 0);
+        gathers(U, &p.tq, bar, sQ + i * kQBytes, U.q0 + i * 2 * kTile + static_cast<int>(rank) * kTile, 64, 2,
+                kTile * 128, 0);
         ++q_use[i];
       }
       for (int j = 0; ok && j < U.nkv; ++j) {
-        stage(U, j * kTile);
         const int ns = pair_ns(U, j);
         const int half = ns >> 1;
         for (int kv = 0; kv < 2; ++kv) {
@@ -757,9 +780,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           __syncwarp();
           uint8_t* dst = sRing + slot * kPairHalfTileBytes;
           if (kv == 0)   // K: keys [rank*half, rank*half + half), both column blocks
-            gathers(&p.tk, bar, dst, (static_cast<int>(rank) * half) >> 2, (half >> 2) * 2, 2, 64 * 128, 0);
+            gathers(U, &p.tk, bar, dst, j * kTile + static_cast<int>(rank) * half, (half >> 2) * 2, 2, 64 * 128, 0);
           else           // V: keys [0, ns), the column block of this CTA's half of d
-            gathers(&p.tv, bar, dst, 0, ns >> 2, 1, 0, 64 * static_cast<int>(rank));
+            gathers(U, &p.tv, bar, dst, j * kTile, ns >> 2, 1, 0, 64 * static_cast<int>(rank));
           ++ld;
         }
       }
