@@ -59,16 +59,33 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
-// Waits for the phase with the given parity to complete, for at most
+// Longest single sleep of a bounded wait before it re-checks its time limit.
+constexpr uint32_t kWaitSleepHintNs = 1000000;
+
+// try_wait with a suspend-time hint: the thread sleeps until the phase
+// completes or about `hint_ns` nanoseconds pass, instead of spinning (a
+// spinning warp takes issue slots from the warps sharing its scheduler).
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+// Waits for the phase with the given parity to complete, for at most about
 // `limit_ns` nanoseconds.  Returns false on timeout (the caller records it).
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
                                                   uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
+  const uint32_t hint = limit_ns < kWaitSleepHintNs ? static_cast<uint32_t>(limit_ns) : kWaitSleepHintNs;
   while (true) {
-    #pragma unroll 1
-    for (int i = 0; i < 64; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, hint)) return true;
     if (globaltimer_ns() - t0 > limit_ns) return false;
   }
 }

@@ -7,11 +7,10 @@
 //  * the row maximum uses 3-input max instructions in eight independent
 //    chains, so it is not one 128-long dependency chain;
 //  * scaling, sums and the polynomial use packed f32x2 FMA/ADD instructions;
-//  * a quarter of the exponentials are evaluated on the FMA pipe as
-//    2^j * p(f), j = round(y), f = y - j, with p the degree-3 minimax fit of
+//  * exponentials run on the MUFU ex2 unit; an FMA-pipe alternative,
+//    2^j * p(f) with j = round(y), f = y - j and p the degree-3 minimax fit of
 //    2^f on [-1/2, 1/2] (coefficients from fit_exp2.py, relative error 7.5e-5,
-//    far below bf16's 2^-8), the rest on the MUFU ex2 unit, so the two
-//    units share the load.
+//    far below bf16's 2^-8), can take a share of them (SWATTN_POLY_SEL).
 #pragma once
 
 #include <stdint.h>
@@ -28,6 +27,14 @@ constexpr float kExp2C3 = 0.0551716685295105f;
 // Adding 1.5 * 2^23 rounds a float of magnitude < 2^22 to the nearest integer,
 // which then sits in the low mantissa bits of the sum.
 constexpr float kRoundMagic = 12582912.0f;
+// Which element pairs (index i of 16 per 32-column chunk) take the FMA-pipe
+// exponential instead of MUFU ex2.  Measured on B200 the softmax is bound by
+// instruction issue, not by MUFU throughput, so the cheaper MUFU path is used
+// for every pair; the polynomial stays available (and tested) for a kernel
+// that is MUFU-bound, e.g. by defining this as ((i) & 3) == 3.
+#ifndef SWATTN_POLY_SEL
+#define SWATTN_POLY_SEL(i) false
+#endif
 
 __device__ __forceinline__ float fmax3f(float a, float b, float c) {
   float d;
@@ -38,20 +45,16 @@ __device__ __forceinline__ float fmax3f(float a, float b, float c) {
 // (d0, d1) = (a0 * b0 + c0, a1 * b1 + c1) in one packed instruction.
 __device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b0, float b1,
                                       float c0, float c1) {
-  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
-      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
-      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-      : "=f"(d0), "=f"(d1)
-      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+  const float2 d = __ffma2_rn(make_float2(a0, a1), make_float2(b0, b1), make_float2(c0, c1));
+  d0 = d.x;
+  d1 = d.y;
 }
 
 // (d0, d1) = (a0 + b0, a1 + b1) in one packed instruction.
 __device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
-  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
-      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-      : "=f"(d0), "=f"(d1)
-      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+  const float2 d = __fadd2_rn(make_float2(a0, a1), make_float2(b0, b1));
+  d0 = d.x;
+  d1 = d.y;
 }
 
 // 2^y for a pair, on the FMA and integer pipes.  y is clamped below at -125
@@ -107,7 +110,7 @@ __device__ __forceinline__ float softmax_tile_to_p(const float (&x)[128], int nc
         const int col = c * 32 + 2 * i;
         float y0, y1, p0, p1;
         ffma2(y0, y1, x[col], x[col + 1], sl2, sl2, neg_m, neg_m);
-        if ((i & 3) == 3) {
+        if (SWATTN_POLY_SEL(i)) {
           exp2_poly2(y0, y1, p0, p1);
         } else {
           p0 = ex2_approx(y0);
