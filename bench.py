@@ -453,6 +453,21 @@ def run_native(args):
             extras["speedup_frac_of_theoretical"] = head[0]["speedup_frac_of_theoretical"]
             extras["full_attention_ms"] = head[0]["ms_full"]
         del flush
+        # An L-layer stack under the interleaved shift schedule (one forward per
+        # layer, layer l shifted by the schedule's Delta_l).
+        if args.schedule_layers > 0:
+            shifts = sw.shift_schedule(args.schedule_layers, wl.win)
+
+            def stack():
+                for shift in shifts:
+                    sw.swattn_fwd(q, k, v, wl.grid, wl.win, shift, wl.scale, out=out, stream=stream)
+            time_launches(stack, 2, stream)
+            ms_stack = statistics.median(time_launches(stack, 10, stream))
+            extras["schedule"] = {
+                "layers": len(shifts), "shifts_thw": [list(x) for x in shifts],
+                "ms_per_stack": ms_stack, "ms_per_layer": ms_stack / len(shifts),
+                "tflops": f_layer * len(shifts) / ms_stack / 1e9,
+                "step_offset": [0, 0, 0]}
         # CPU baseline: the oracle on a bounded sample of the same workload
         if not args.no_cpu_baseline:
             qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
@@ -505,6 +520,8 @@ def main():
     ap.add_argument("--no-sweep", action="store_true", help="skip the per-workload table")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end timing")
+    ap.add_argument("--schedule-layers", type=int, default=8,
+                    help="also time an L-layer stack under the interleaved shift schedule (0: off)")
     ap.add_argument("--workload", default=HEADLINE,
                     help="workload name from shifted_window_attention_swattn_b200.inputs "
                          "(profiling runs of a smaller case; the default is the headline)")

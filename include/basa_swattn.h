@@ -93,6 +93,23 @@ int basa_swattn_flops(int B, int heads, int T, int H, int W, int d, const int wi
                       double* flops);
 
 /*
+ * The per-layer window offsets of the interleaved shift schedule
+ * (§3.1 "Interleaved shift schedule"), per axis a with window w = win[a]:
+ *   delta = max(1, floor(w / L)),  a_i = (i * delta) mod w  for i = 0..L-1,
+ *   b = (a_0, a_K, a_1, a_{K+1}, ...)  with K = ceil(L / 2)  (the first and
+ *        second halves of a interleaved; for odd L the first half has the
+ *        extra element, which comes last),
+ *   shift[l][a] = (b_l + step_offset[a]) mod w.
+ * step_offset is the denoising-step term c_s of the schedule (the pages leave
+ * its values open; pass zeros for a step-independent schedule).
+ * shifts: host array of L * 3 ints, written as [l][t, h, w]; each entry is a
+ * value for basa_swattn_fwd's `shift` argument.  An axis whose window spans
+ * the whole grid may be given any shift: it does not change the result.
+ * Returns BASA_ERR_INVALID_ARG for L < 1, a window < 1 or null pointers.
+ */
+int basa_shift_schedule(int L, const int win[3], const int step_offset[3], int* shifts);
+
+/*
  * Synchronises `stream`, then returns BASA_ERR_DEVICE if any launch since the
  * previous call gave up on a bounded wait (BASA_OK otherwise), and clears the
  * record.  Also returns BASA_ERR_CUDA if the synchronisation itself fails.

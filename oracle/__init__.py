@@ -152,3 +152,36 @@ def flops(B, heads, T, H, W, d, win) -> float:
     lib = _load()
     w3 = _I3(*[int(a) for a in win])
     return float(lib.oref_flops(int(B), int(heads), int(T), int(H), int(W), int(d), w3))
+
+
+def shift_schedule(L, win, step_offset=(0, 0, 0)):
+    """Interleaved shift schedule, §3.1 "Interleaved shift schedule", taken step
+    by step in the pages' order for each axis with window w:
+
+      delta = max(1, floor(w / L));  a_i = (i * delta) mod w, i = 0..L-1;
+      b = (a_0, a_K, a_1, a_{K+1}, ..., a_{K-1}, a_{L-1}): the halves
+          a_0..a_{K-1} and a_K..a_{L-1} interleaved, first half first;
+      Delta_l = (b_l + c_s) mod w.
+
+    Readings: K = ceil(L / 2) (the pages do not define K; this is the value for
+    which the printed sequence ends with a_{K-1}, a_{L-1} when L is even), and
+    for odd L the first half's extra element a_{K-1} comes last.  c_s, the
+    denoising-step offset, is an input (the pages leave its values open).
+    Returns a list of L (t, h, w) triples.
+    """
+    L = int(L)
+    if L < 1 or len(win) != 3 or min(win) < 1:
+        raise ValueError("L and the window extents must be >= 1")
+    K = -(-L // 2)
+    per_axis = []
+    for w, c in zip(win, step_offset):
+        delta = max(1, w // L)
+        a = [(i * delta) % w for i in range(L)]
+        first, second = a[:K], a[K:]
+        b = []
+        for i in range(K):
+            b.append(first[i])
+            if i < len(second):
+                b.append(second[i])
+        per_axis.append([(x + c) % w for x in b])
+    return [tuple(per_axis[ax][l] for ax in range(3)) for l in range(L)]

@@ -16,7 +16,7 @@ import os
 import threading
 
 __all__ = [
-    "swattn_fwd", "swattn_fwd_from_host", "index_map", "index_map_host", "flops",
+    "swattn_fwd", "swattn_fwd_from_host", "index_map", "index_map_host", "flops", "shift_schedule",
     "last_device_error", "set_wait_timeout_ns", "strerror", "library_path", "SwattnError",
 ]
 
@@ -65,6 +65,8 @@ def _load():
         lib.basa_swattn_index_map_host.restype = ci
         lib.basa_swattn_flops.argtypes = [ci] * 6 + [_I3, ctypes.POINTER(ctypes.c_double)]
         lib.basa_swattn_flops.restype = ci
+        lib.basa_shift_schedule.argtypes = [ci, _I3, _I3, vp]
+        lib.basa_shift_schedule.restype = ci
         lib.basa_swattn_last_device_error.argtypes = [vp]
         lib.basa_swattn_last_device_error.restype = ci
         lib.basa_swattn_set_wait_timeout_ns.argtypes = [ctypes.c_ulonglong]
@@ -204,6 +206,22 @@ def flops(B, heads, grid, d, win) -> float:
     if rc != BASA_OK:
         raise SwattnError(rc, "basa_swattn_flops")
     return res.value
+
+
+def shift_schedule(L, win, step_offset=(0, 0, 0)):
+    """Per-layer shifts of the interleaved shift schedule (§3.1): a list of L
+    (t, h, w) triples for layers 0..L-1, each usable as ``swattn_fwd``'s ``shift``.
+    ``step_offset`` is the schedule's denoising-step term c_s."""
+    lib = _load()
+    w3, c3 = _triple(win, "win"), _triple(step_offset, "step_offset")
+    L = int(L)
+    if L < 1:
+        raise SwattnError(BASA_ERR_INVALID_ARG, "basa_shift_schedule")
+    out = (ctypes.c_int * (3 * L))()
+    rc = lib.basa_shift_schedule(L, _I3(*w3), _I3(*c3), ctypes.cast(out, ctypes.c_void_p))
+    if rc != BASA_OK:
+        raise SwattnError(rc, "basa_shift_schedule")
+    return [tuple(out[3 * l:3 * l + 3]) for l in range(L)]
 
 
 def last_device_error(stream=None) -> int:

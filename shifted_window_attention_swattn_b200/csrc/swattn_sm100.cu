@@ -1240,6 +1240,27 @@ extern "C" int basa_swattn_flops(int B, int heads, int T, int H, int W, int d, c
   return BASA_OK;
 }
 
+extern "C" int basa_shift_schedule(int L, const int win[3], const int step_offset[3], int* shifts) {
+  if (L < 1 || !win || !step_offset || !shifts) return BASA_ERR_INVALID_ARG;
+  for (int a = 0; a < 3; ++a)
+    if (win[a] < 1) return BASA_ERR_INVALID_ARG;
+  const int K = (L + 1) / 2;
+  for (int a = 0; a < 3; ++a) {
+    const long long w = win[a];
+    const long long delta = w / L > 1 ? w / L : 1;
+    long long c = step_offset[a] % w;
+    if (c < 0) c += w;
+    for (int l = 0; l < L; ++l) {
+      // b_l: even positions take a_0, a_1, ... (first half), odd positions
+      // a_K, a_{K+1}, ... (second half).
+      const long long i = (l % 2 == 0) ? l / 2 : K + l / 2;
+      const long long b = (i * delta) % w;
+      shifts[3 * l + a] = static_cast<int>((b + c) % w);
+    }
+  }
+  return BASA_OK;
+}
+
 extern "C" int basa_swattn_last_device_error(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return BASA_ERR_CUDA;
   int v = 0;

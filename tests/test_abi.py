@@ -129,3 +129,20 @@ def test_python_binding_rejects_non_cuda_tensors(lib):
     q = torch.zeros(1, 16, 1, 64, dtype=torch.bfloat16)
     with pytest.raises(TypeError):
         sw.swattn_fwd(q, q, q, (1, 4, 4), (1, 2, 2), (0, 0, 0))
+
+
+def test_shift_schedule_equals_oracle(lib):
+    for L in (1, 2, 3, 5, 8, 19, 57):
+        for win in ((1, 16, 16), (7, 15, 16), (7, 10, 13), (21, 1, 32), (3, 4, 300)):
+            for off in ((0, 0, 0), (1, 5, -3), (-8, 40, 7)):
+                assert sw.shift_schedule(L, win, off) == oracle.shift_schedule(L, win, off), (L, win, off)
+
+
+def test_shift_schedule_argument_errors(lib):
+    out = (ctypes.c_int * 30)()
+    z = I3(0, 0, 0)
+    assert lib.basa_shift_schedule(0, I3(1, 8, 8), z, ctypes.cast(out, ctypes.c_void_p)) == sw.BASA_ERR_INVALID_ARG
+    assert lib.basa_shift_schedule(4, I3(1, 0, 8), z, ctypes.cast(out, ctypes.c_void_p)) == sw.BASA_ERR_INVALID_ARG
+    assert lib.basa_shift_schedule(4, I3(1, 8, 8), z, None) == sw.BASA_ERR_INVALID_ARG
+    with pytest.raises(sw.SwattnError):
+        sw.shift_schedule(0, (1, 8, 8))

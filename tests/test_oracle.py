@@ -246,3 +246,55 @@ def test_masked_attention_helper_is_itself_sane():
         masked_window_attention(q, k, v, T, H, W, (T, H, W), (0, 0, 0), 0.5), full, atol=0)
     np.testing.assert_allclose(
         masked_window_attention(q, k, v, T, H, W, (1, 1, 1), (0, 1, 2), 0.5), v, atol=0)
+
+
+# ---------------------------------------------------------------- shift schedule
+# §3.1 "Interleaved shift schedule": delta = max(1, floor(w/L)), a_i = (i delta) mod w,
+# b = (a_0, a_K, a_1, a_{K+1}, ...), Delta_l = (b_l + c_s) mod w.  Values below are
+# worked by hand from that definition.
+
+@pytest.mark.parametrize("L,w,expected", [
+    (8, 16, [0, 8, 2, 10, 4, 12, 6, 14]),     # delta 2, K 4
+    (4, 16, [0, 8, 4, 12]),                   # delta 4, K 2
+    (5, 7, [0, 3, 1, 4, 2]),                  # delta 1, K 3: odd L, a_{K-1} last
+    (6, 4, [0, 3, 1, 0, 2, 1]),               # L > w: delta 1, a wraps mod w
+    (3, 32, [0, 20, 10]),                     # delta 10, K 2
+    (1, 9, [0]),
+])
+def test_shift_schedule_hand_worked(L, w, expected):
+    sched = oracle.shift_schedule(L, (1, w, w))
+    assert [s[1] for s in sched] == expected
+    assert [s[2] for s in sched] == expected
+    assert all(s[0] == 0 for s in sched)      # a window of one along t: only shift 0
+
+
+def test_shift_schedule_two_layers_is_the_swin_alternation():
+    # L = 2 gives delta = floor(w/2) and b = (0, floor(w/2)): Swin's alternating half shift
+    for w in (7, 8, 13, 16, 32):
+        assert oracle.shift_schedule(2, (w, w, w)) == [(0, 0, 0), (w // 2,) * 3]
+
+
+def test_shift_schedule_step_offset_and_range():
+    assert [s[1] for s in oracle.shift_schedule(2, (1, 16, 16), (0, 5, -3))] == [5, 13]
+    assert [s[2] for s in oracle.shift_schedule(2, (1, 16, 16), (0, 5, -3))] == [13, 5]
+    for L in range(1, 12):
+        for w in (1, 3, 8, 15, 16):
+            sched = oracle.shift_schedule(L, (w, w, w), (L, -L, 2 * L))
+            assert all(0 <= x < w for s in sched for x in s)
+
+
+def test_shift_schedule_is_a_permutation_of_the_offsets():
+    # b reorders a: same multiset, every layer present once
+    for L in range(1, 20):
+        for w in (4, 13, 16, 32):
+            delta = max(1, w // L)
+            a = sorted((i * delta) % w for i in range(L))
+            b = sorted(s[1] for s in oracle.shift_schedule(L, (1, w, 1)))
+            assert a == b
+
+
+def test_shift_schedule_rejects_bad_arguments():
+    with pytest.raises(ValueError):
+        oracle.shift_schedule(0, (1, 8, 8))
+    with pytest.raises(ValueError):
+        oracle.shift_schedule(4, (1, 0, 8))

@@ -192,3 +192,19 @@ def test_full_attention_mode_sampled(wl):
                              wl.scale, tri)
     got = out[tri[:, 0], tri[:, 1], tri[:, 2]].float().cpu().numpy()
     _check(got, ref, "full attention")
+
+
+@pytest.mark.parametrize("d,grid,win,L", [
+    (128, (1, 24, 24), (1, 8, 8), 4),       # 2D, every layer of a 4-layer schedule
+    (64, (3, 12, 10), (2, 6, 5), 3),        # 3D, truncated windows along t
+    (128, (2, 9, 20), (2, 9, 7), 5),        # odd L, truncated along w
+])
+def test_shift_schedule_layers(d, grid, win, L):
+    # every layer of the interleaved shift schedule, through the kernel, against the oracle
+    T, H, W = grid
+    q, k, v = make_custom(1, 2, d, T, H, W, seed=L)
+    scale = 1.0 / math.sqrt(d)
+    for shift in sw.shift_schedule(L, win, (0, 1, 2)):
+        out = _run_gpu(q, k, v, grid, win, shift, scale).float().cpu().numpy()
+        ref = oracle.swattn_fwd(q, k, v, 1, 2, T, H, W, d, win, shift, scale)
+        _check(out, ref, f"schedule layer shift={shift}")
