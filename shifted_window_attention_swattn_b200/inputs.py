@@ -13,6 +13,7 @@ Recipe (every workload):
     the workload's seed, in the order Q, K, V, then rounded to bf16;
   * layout [B, T*H*W, heads, d], raster token order (t, h, w);
   * scale = 1/sqrt(d);
+  * seed = the workload's index in WORKLOADS;
   * the 4096^2 FLUX-like workload then draws one factor s_h ~ U(0.5, 2) per
     head and multiplies that head's Q and K rows by it (in fp32, before the
     bf16 rounding), so logits of head h have standard deviation s_h^2.
@@ -67,6 +68,14 @@ WORKLOADS = (
              ((0, 0, 0), (3, 5, 6)), 3),
     Workload("wan-720p-21x45x80-w7x15x16", 1, 40, 128, 21, 45, 80, (7, 15, 16),
              ((0, 0, 0), (3, 7, 8)), 4),
+    # The pages' own Wan2.1 geometry (a 1664x960, 81-frame video: latent grid
+    # 21 x 60 x 104, 12 heads of 128), with the pages' spatial-only windows that
+    # keep the full temporal extent: 15 x 26 (8,190 tokens) and the
+    # non-divisible 10 x 10 (the last window along w holds 4 columns).
+    Workload("wan-pages-21x60x104-w21x15x26", 1, 12, 128, 21, 60, 104, (21, 15, 26),
+             ((0, 0, 0), (0, 7, 13)), 5),
+    Workload("wan-pages-21x60x104-w21x10x10", 1, 12, 128, 21, 60, 104, (21, 10, 10),
+             ((0, 0, 0), (0, 5, 5)), 6),
 )
 
 BY_NAME = {w.name: w for w in WORKLOADS}
