@@ -132,4 +132,36 @@ __device__ __forceinline__ float softmax_tile_to_p(const float (&x)[128], int nc
   return (s0 + s1) + (s2 + s3);
 }
 
+// P for half h of a 128-column S row in registers (columns 64h .. 64h+63):
+// 32 packed bf16 pairs in pk (pk[i] holds columns 64h+2i, 64h+2i+1), for one
+// 32-column TMEM store.  Returns the fp32 sum.  kPartial: columns >= kv_valid
+// are padding keys (P = 0).
+template <bool kPartial, int kHalf>
+__device__ __forceinline__ float softmax_half_to_pk(const float (&x)[128], int kv_valid, float sl2,
+                                                    float neg_m, uint32_t (&pk)[32]) {
+  float s0 = 0.0f, s1 = 0.0f, s2 = 0.0f, s3 = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const int col = 64 * kHalf + 2 * i;
+    float y0, y1, p0, p1;
+    ffma2(y0, y1, x[col], x[col + 1], sl2, sl2, neg_m, neg_m);
+    if (SWATTN_POLY_SEL(i & 15)) {
+      exp2_poly2(y0, y1, p0, p1);
+    } else {
+      p0 = ex2_approx(y0);
+      p1 = ex2_approx(y1);
+    }
+    if (kPartial) {
+      p0 = col < kv_valid ? p0 : 0.0f;
+      p1 = col + 1 < kv_valid ? p1 : 0.0f;
+    }
+    if (i & 1)
+      fadd2(s2, s3, s2, s3, p0, p1);
+    else
+      fadd2(s0, s1, s0, s1, p0, p1);
+    pk[i] = pack_bf16x2(p0, p1);
+  }
+  return (s0 + s1) + (s2 + s3);
+}
+
 }  // namespace swattn

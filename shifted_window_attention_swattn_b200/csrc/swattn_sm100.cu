@@ -906,21 +906,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         ++s_use;
         tc_fence_after();
         const int kvv = kv_valid_of(U, j);
-        const int nchunks = (kvv + 31) >> 5;
+        // The whole S row in one TMEM load and P in two 32-column stores, so S
+        // and P each sit in one contiguous run of registers; columns past the
+        // tile's keys (last tile of a window) are masked, not skipped.
         float x[kTile];
+        {
+          uint32_t r[kTile];
+          tmem_ld128(tS, r);
+          tmem_wait_ld();
+          tmem_tie(r);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          if (c < nchunks) {
-            uint32_t r[32];
-            tmem_ld32(tS + c * 32, r);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) x[c * 32 + i] = __uint_as_float(r[i]);
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) x[c * 32 + i] = -INFINITY;
-          }
+          for (int i = 0; i < kTile; ++i) x[i] = __uint_as_float(r[i]);
         }
-        tmem_wait_ld();
         if (kvv < kTile) {
 #pragma unroll
           for (int i = 0; i < kTile; ++i)
@@ -935,8 +932,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           m_run = m_new;
         }
         const float neg_m = -m_run;
-        const float rowsum = kvv < kTile ? softmax_tile_to_p<true>(x, nchunks, kvv, sl2, neg_m, tS)
-                                         : softmax_tile_to_p<false>(x, nchunks, kvv, sl2, neg_m, tS);
+        float rowsum;
+        {
+          uint32_t pk[32];
+          rowsum = kvv < kTile ? softmax_half_to_pk<true, 0>(x, kvv, sl2, neg_m, pk)
+                               : softmax_half_to_pk<false, 0>(x, kvv, sl2, neg_m, pk);
+          tmem_st32(tS, pk);
+          rowsum += kvv < kTile ? softmax_half_to_pk<true, 1>(x, kvv, sl2, neg_m, pk)
+                                : softmax_half_to_pk<false, 1>(x, kvv, sl2, neg_m, pk);
+          tmem_st32(tS + 32, pk);
+        }
         l_run = l_run * alpha + rowsum;
         if (j > 0 && __any_sync(0xffffffffu, need)) {
           for (int c = 0; c < 4; ++c) {
