@@ -92,46 +92,6 @@ __device__ __forceinline__ float row_max128(const float (&x)[128]) {
   return fmax3f(fmax3f(m[0], m[1], m[2]), fmax3f(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
 }
 
-// P = 2^(x * sl2 - m) for one S row in registers, packed to bf16 pairs and
-// stored over the front of the S row in TMEM at tS (32 columns of S become 16
-// columns of bf16 pairs).  Returns the fp32 row sum.  kPartial: columns
-// >= kv_valid are padding keys and get P = 0.  nchunks: 32-column chunks to
-// produce (those the P V product reads).
-template <bool kPartial>
-__device__ __forceinline__ float softmax_tile_to_p(const float (&x)[128], int nchunks, int kv_valid,
-                                                   float sl2, float neg_m, uint32_t tS) {
-  float s0 = 0.0f, s1 = 0.0f, s2 = 0.0f, s3 = 0.0f;
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    if (c < nchunks) {
-      uint32_t pk[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int col = c * 32 + 2 * i;
-        float y0, y1, p0, p1;
-        ffma2(y0, y1, x[col], x[col + 1], sl2, sl2, neg_m, neg_m);
-        if (SWATTN_POLY_SEL(i)) {
-          exp2_poly2(y0, y1, p0, p1);
-        } else {
-          p0 = ex2_approx(y0);
-          p1 = ex2_approx(y1);
-        }
-        if (kPartial) {
-          p0 = col < kv_valid ? p0 : 0.0f;
-          p1 = col + 1 < kv_valid ? p1 : 0.0f;
-        }
-        if (i & 1)
-          fadd2(s2, s3, s2, s3, p0, p1);
-        else
-          fadd2(s0, s1, s0, s1, p0, p1);
-        pk[i] = pack_bf16x2(p0, p1);
-      }
-      tmem_st16(tS + c * 16, pk);
-    }
-  }
-  return (s0 + s1) + (s2 + s3);
-}
-
 // P for half h of a 128-column S row in registers (columns 64h .. 64h+63):
 // 32 packed bf16 pairs in pk (pk[i] holds columns 64h+2i, 64h+2i+1), for one
 // 32-column TMEM store.  Returns the fp32 sum.  kPartial: columns >= kv_valid

@@ -262,6 +262,49 @@ __device__ __forceinline__ void unit_rows4(const Geometry& g, const Unit& U, int
   }
 }
 
+// One key step of the online softmax for the S row of this thread at TMEM
+// address tS (128 fp32 columns): the row maximum against the running maximum
+// m_run (updated only when it grows by more than kRescaleThreshold; then alpha
+// = 2^(m_old - m_new) and need is set), P = 2^(S*sl2 - m_run) in bf16 written
+// back over the front of the row, and the fp32 sum of P returned.  The whole
+// row comes in one TMEM load and P goes out in two 32-column stores, so S and
+// P each sit in one contiguous run of registers; columns >= kv_valid (the last
+// tile of a window) are masked, not skipped.
+__device__ __forceinline__ float softmax_row_step(uint32_t tS, int kv_valid, float sl2, float& m_run,
+                                                  float& alpha, bool& need) {
+  float x[kTile];
+  {
+    uint32_t r[kTile];
+    tmem_ld128(tS, r);
+    tmem_wait_ld();
+    tmem_tie(r);
+#pragma unroll
+    for (int i = 0; i < kTile; ++i) x[i] = __uint_as_float(r[i]);
+  }
+  if (kv_valid < kTile) {
+#pragma unroll
+    for (int i = 0; i < kTile; ++i)
+      if (i >= kv_valid) x[i] = -INFINITY;
+  }
+  const float mx = row_max128(x);
+  const float m_new = fmaxf(m_run, mx * sl2);
+  need = m_new > m_run + kRescaleThreshold;
+  alpha = 1.0f;
+  if (need) {
+    alpha = ex2_approx(m_run - m_new);
+    m_run = m_new;
+  }
+  const float neg_m = -m_run;
+  uint32_t pk[32];
+  float rowsum = kv_valid < kTile ? softmax_half_to_pk<true, 0>(x, kv_valid, sl2, neg_m, pk)
+                                  : softmax_half_to_pk<false, 0>(x, kv_valid, sl2, neg_m, pk);
+  tmem_st32(tS, pk);
+  rowsum += kv_valid < kTile ? softmax_half_to_pk<true, 1>(x, kv_valid, sl2, neg_m, pk)
+                             : softmax_half_to_pk<false, 1>(x, kv_valid, sl2, neg_m, pk);
+  tmem_st32(tS + 32, pk);
+  return rowsum;
+}
+
 // S_i (+)= Q_i K^T over the head dimension: d/16 MMAs of M=128, N=n_s, K=16.
 __device__ __forceinline__ void issue_qk(uint32_t tmem_s, uint32_t q_addr, uint32_t k_addr, int d,
                                          int n_s) {
@@ -484,38 +527,9 @@ __global__ void __launch_bounds__(kThreads, 1) swattn_fwd_kernel(const __grid_co
         if (!ok) break;
         ++s_use;
         tc_fence_after();
-        const int kvv = kv_valid_of(U, j);
-        const int nchunks = (kvv + 31) >> 5;
-        float x[kTile];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          if (c < nchunks) {
-            uint32_t r[32];
-            tmem_ld32(tS + c * 32, r);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) x[c * 32 + i] = __uint_as_float(r[i]);
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) x[c * 32 + i] = -INFINITY;
-          }
-        }
-        tmem_wait_ld();
-        if (kvv < kTile) {
-#pragma unroll
-          for (int i = 0; i < kTile; ++i)
-            if (i >= kvv) x[i] = -INFINITY;
-        }
-        const float mx = row_max128(x);
-        const float m_new = fmaxf(m_run, mx * sl2);
-        const bool need = m_new > m_run + kRescaleThreshold;
-        float alpha = 1.0f;
-        if (need) {
-          alpha = ex2_approx(m_run - m_new);
-          m_run = m_new;
-        }
-        const float neg_m = -m_run;
-        const float rowsum = kvv < kTile ? softmax_tile_to_p<true>(x, nchunks, kvv, sl2, neg_m, tS)
-                                         : softmax_tile_to_p<false>(x, nchunks, kvv, sl2, neg_m, tS);
+        float alpha;
+        bool need;
+        const float rowsum = softmax_row_step(tS, kv_valid_of(U, j), sl2, m_run, alpha, need);
         l_run = l_run * alpha + rowsum;
         if (j > 0 && __any_sync(0xffffffffu, need)) {
           // O_i holds P V of tiles 0..j-1 (complete: S_i(j) was issued after
@@ -905,43 +919,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         if (!ok) break;
         ++s_use;
         tc_fence_after();
-        const int kvv = kv_valid_of(U, j);
-        // The whole S row in one TMEM load and P in two 32-column stores, so S
-        // and P each sit in one contiguous run of registers; columns past the
-        // tile's keys (last tile of a window) are masked, not skipped.
-        float x[kTile];
-        {
-          uint32_t r[kTile];
-          tmem_ld128(tS, r);
-          tmem_wait_ld();
-          tmem_tie(r);
-#pragma unroll
-          for (int i = 0; i < kTile; ++i) x[i] = __uint_as_float(r[i]);
-        }
-        if (kvv < kTile) {
-#pragma unroll
-          for (int i = 0; i < kTile; ++i)
-            if (i >= kvv) x[i] = -INFINITY;
-        }
-        const float mx = row_max128(x);
-        const float m_new = fmaxf(m_run, mx * sl2);
-        const bool need = m_new > m_run + kRescaleThreshold;
-        float alpha = 1.0f;
-        if (need) {
-          alpha = ex2_approx(m_run - m_new);
-          m_run = m_new;
-        }
-        const float neg_m = -m_run;
-        float rowsum;
-        {
-          uint32_t pk[32];
-          rowsum = kvv < kTile ? softmax_half_to_pk<true, 0>(x, kvv, sl2, neg_m, pk)
-                               : softmax_half_to_pk<false, 0>(x, kvv, sl2, neg_m, pk);
-          tmem_st32(tS, pk);
-          rowsum += kvv < kTile ? softmax_half_to_pk<true, 1>(x, kvv, sl2, neg_m, pk)
-                                : softmax_half_to_pk<false, 1>(x, kvv, sl2, neg_m, pk);
-          tmem_st32(tS + 32, pk);
-        }
+        float alpha;
+        bool need;
+        const float rowsum = softmax_row_step(tS, kv_valid_of(U, j), sl2, m_run, alpha, need);
         l_run = l_run * alpha + rowsum;
         if (j > 0 && __any_sync(0xffffffffu, need)) {
           for (int c = 0; c < 4; ++c) {
