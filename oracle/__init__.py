@@ -6,7 +6,8 @@ path (``shifted_window_attention_swattn_b200``) never imports it and shares no
 code with it.
 
 The arithmetic lives in ``ref_swattn.c`` (plain C, fp64, one materialised array
-per stage).  This module only builds that file with gcc and marshals arguments
+per stage), including the pooled global memory of §3.2 ("K/V-Pooled Global
+Memory").  This module only builds that file with gcc and marshals arguments
 through ctypes.  Method: "Backend-Agnostic Sparse Attention for Fast
 High-Resolution Visual Generation" (BASA), §3.1 "Shifted Window Sparse
 Attention" and Appendix A.1 "Regular execution with standard attention
@@ -58,6 +59,12 @@ def _load():
             lib.oref_swattn_rows.restype = ctypes.c_int
             lib.oref_flops.argtypes = [ctypes.c_int] * 6 + [_I3]
             lib.oref_flops.restype = ctypes.c_double
+            lib.oref_swattn_fwd_mem.argtypes = (
+                [ctypes.c_void_p] * 5 + [ctypes.c_int, ctypes.c_void_p] + [ctypes.c_int] * 6
+                + [_I3, _I3, ctypes.c_double] + [ctypes.c_int] * 3)
+            lib.oref_swattn_fwd_mem.restype = ctypes.c_int
+            lib.oref_kv_pool.argtypes = [ctypes.c_void_p, ctypes.c_void_p] + [ctypes.c_int] * 6 + [_I3]
+            lib.oref_kv_pool.restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -152,6 +159,61 @@ def flops(B, heads, T, H, W, d, win) -> float:
     lib = _load()
     w3 = _I3(*[int(a) for a in win])
     return float(lib.oref_flops(int(B), int(heads), int(T), int(H), int(W), int(d), w3))
+
+
+def n_pooled(T, H, W, pool) -> int:
+    """Pooled memory tokens G = prod ceil(n_a / p_a) (§3.2; truncated last patches)."""
+    n = 1
+    for ext, p in zip((T, H, W), pool):
+        if int(p) < 1 or int(ext) < 1:
+            raise ValueError("grid and pooling extents must be >= 1")
+        n *= -(-int(ext) // int(p))
+    return n
+
+
+def kv_pool(x, B, heads, T, H, W, d, pool):
+    """fp64 [B, G, heads, d]: means of x (bf16 [B, T*H*W, heads, d]) over the
+    p_t x p_h x p_w patches of the unshifted grid, patches in raster order (§3.2)."""
+    lib = _load()
+    xb = _bits(x)
+    G = n_pooled(T, H, W, pool)
+    out = np.empty((int(B), G, int(heads), int(d)), dtype=np.float64)
+    rc = lib.oref_kv_pool(xb.ctypes.data, out.ctypes.data, int(B), int(heads), int(T), int(H),
+                          int(W), int(d), _I3(*[int(a) for a in pool]))
+    if rc != 0:
+        raise ValueError(f"oref_kv_pool failed ({rc})")
+    return out
+
+
+def round_to_bf16_bits(x) -> np.ndarray:
+    """Round fp64 values to bf16 (round to nearest, ties to even) as uint16 bits."""
+    f = np.ascontiguousarray(np.asarray(x, dtype=np.float64).astype(np.float32))
+    u = f.view(np.uint32).astype(np.uint64)
+    lsb = (u >> 16) & 1
+    return ((u + 0x7FFF + lsb) >> 16).astype(np.uint16)
+
+
+def swattn_fwd_mem(q, k, v, kx, vx, E, B, heads, T, H, W, d, win, shift, scale, nthreads=None):
+    """fp64 [B, T*H*W, heads, d]: the shifted-window forward where every window's
+    keys and values are extended by the E extra tokens kx, vx (bf16 [B, E, heads, d])
+    of its (b, head): K^mem = [K_W; K_x], V^mem = [V_W; V_x] (§3.2)."""
+    lib = _load()
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    kxb, vxb = _bits(kx), _bits(vx)
+    N = int(T) * int(H) * int(W)
+    if kxb.size != int(B) * int(E) * int(heads) * int(d) or vxb.size != kxb.size:
+        raise ValueError("kx/vx must hold B*E*heads*d elements")
+    if nthreads is None:
+        nthreads = max(1, len(os.sched_getaffinity(0)))
+    out = np.full((int(B), N, int(heads), int(d)), np.nan, dtype=np.float64)
+    w3, s3 = _geom_args(win, shift)
+    rc = lib.oref_swattn_fwd_mem(qb.ctypes.data, kb.ctypes.data, vb.ctypes.data, kxb.ctypes.data,
+                                 vxb.ctypes.data, int(E), out.ctypes.data, int(B), int(heads),
+                                 int(T), int(H), int(W), int(d), w3, s3, float(scale), 0,
+                                 int(heads), int(nthreads))
+    if rc != 0:
+        raise ValueError(f"oref_swattn_fwd_mem failed ({rc})")
+    return out
 
 
 def shift_schedule(L, win, step_offset=(0, 0, 0)):

@@ -41,6 +41,11 @@
  *   - every head and every batch item uses the same partition;
  *   - the inputs are bf16 bit patterns, widened exactly to fp64.
  *
+ *   §3.2 "K/V-Pooled Global Memory": K_bar, V_bar are means of K, V over
+ *   spatial patches of the grid; each window's keys and values become
+ *   [K_W; K_bar] and [V_W; V_bar] (oref_kv_pool builds the means,
+ *   oref_swattn_fwd_mem attends over a window plus any extra segment).
+ *
  * Data layout: Q, K, V are bf16 [B, T*H*W, heads, d] (raster token order t,h,w),
  * passed as uint16 bit patterns; the output is fp64 [B, T*H*W, heads, d].
  */
@@ -210,6 +215,39 @@ static void window_attention(const double *q, const double *k, const double *v, 
     }
 }
 
+/*
+ * The same with an extra segment appended to the window's keys and values
+ * (§3.2 "K/V-Pooled Global Memory": K^mem = [K_W; K_bar], V^mem = [V_W; V_bar]):
+ * keys j < n are the window's, keys n <= j < n + E are kx/vx ([E][d]).
+ * work holds n + E doubles.
+ */
+static void window_attention_mem(const double *q, const double *k, const double *v,
+                                 const double *kx, const double *vx, double *o,
+                                 int n, int E, int d, double scale, double *work)
+{
+    int i, j, c;
+    for (i = 0; i < n; ++i) {
+        double mx = -INFINITY, sum = 0.0;
+        for (j = 0; j < n + E; ++j) {
+            const double *kr = j < n ? k + (long)j * d : kx + (long)(j - n) * d;
+            double s = 0.0;
+            for (c = 0; c < d; ++c) s += q[(long)i * d + c] * kr[c];
+            work[j] = scale * s;
+            if (work[j] > mx) mx = work[j];
+        }
+        for (j = 0; j < n + E; ++j) {
+            work[j] = exp(work[j] - mx);
+            sum += work[j];
+        }
+        for (c = 0; c < d; ++c) o[(long)i * d + c] = 0.0;
+        for (j = 0; j < n + E; ++j) {
+            const double *vr = j < n ? v + (long)j * d : vx + (long)(j - n) * d;
+            double pj = work[j] / sum;
+            for (c = 0; c < d; ++c) o[(long)i * d + c] += pj * vr[c];
+        }
+    }
+}
+
 /* ------------------------------------------------------------------ */
 /* index map: which original token sits in (window, slot)              */
 /* ------------------------------------------------------------------ */
@@ -259,6 +297,8 @@ typedef struct {
     const int *count;
     int d;
     double scale;
+    const double *kx, *vx;      /* extra key/value segment [E][d], or NULL */
+    int E;
     long next;                  /* shared window counter */
     int failed;
 } attn_job_t;
@@ -266,7 +306,7 @@ typedef struct {
 static void *attn_worker(void *arg)
 {
     attn_job_t *job = (attn_job_t *)arg;
-    double *work = (double *)malloc(sizeof(double) * (size_t)job->g->nw_max);
+    double *work = (double *)malloc(sizeof(double) * (size_t)(job->g->nw_max + job->E));
     if (!work) {
         __atomic_store_n(&job->failed, 1, __ATOMIC_SEQ_CST);
         return NULL;
@@ -276,26 +316,34 @@ static void *attn_worker(void *arg)
         long off;
         if (m >= job->g->n_windows) break;
         off = m * job->g->nw_max * job->d;
-        window_attention(job->qw + off, job->kw + off, job->vw + off, job->ow + off,
-                         job->count[m], job->d, job->scale, work);
+        if (job->E > 0)
+            window_attention_mem(job->qw + off, job->kw + off, job->vw + off, job->kx, job->vx,
+                                 job->ow + off, job->count[m], job->E, job->d, job->scale, work);
+        else
+            window_attention(job->qw + off, job->kw + off, job->vw + off, job->ow + off,
+                             job->count[m], job->d, job->scale, work);
     }
     free(work);
     return NULL;
 }
 
 /*
+ * The forward, with an optional extra key/value segment (kxb, vxb: bf16
+ * [B, E, heads, d]; E = 0 for none) appended to every window of its (b, head).
  * out[b, token, head, :] for head in [head_begin, head_end); other heads of
  * out are left untouched.  nthreads <= 0 means one thread.
  */
-int oref_swattn_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, double *out,
-                    int B, int heads, int T, int H, int W, int d,
-                    const int win[3], const int shift[3], double scale,
-                    int head_begin, int head_end, int nthreads)
+static int swattn_fwd_impl(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                           const uint16_t *kxb, const uint16_t *vxb, int E, double *out,
+                           int B, int heads, int T, int H, int W, int d,
+                           const int win[3], const int shift[3], double scale,
+                           int head_begin, int head_end, int nthreads)
 {
     geom_t g;
     long N, wsz, tok, c;
     int b, hd, i, rc;
     double *xq, *xk, *xv, *rq, *rk, *rv, *wq, *wk, *wv, *wo, *ro, *y;
+    double *xkx = NULL, *xvx = NULL;
     int *count;
     rc = geom_init(&g, T, H, W, win, shift);
     if (rc) return rc;
@@ -317,8 +365,13 @@ int oref_swattn_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, dou
     wv = (double *)calloc((size_t)wsz, sizeof(double));
     wo = (double *)calloc((size_t)wsz, sizeof(double));
     count = (int *)malloc(sizeof(int) * (size_t)g.n_windows);
+    if (E > 0) {
+        xkx = (double *)malloc(sizeof(double) * (size_t)E * (size_t)d);
+        xvx = (double *)malloc(sizeof(double) * (size_t)E * (size_t)d);
+    }
     rc = OREF_OK;
-    if (!xq || !xk || !xv || !rq || !rk || !rv || !ro || !y || !wq || !wk || !wv || !wo || !count) {
+    if (!xq || !xk || !xv || !rq || !rk || !rv || !ro || !y || !wq || !wk || !wv || !wo || !count ||
+        (E > 0 && (!xkx || !xvx))) {
         rc = OREF_ERR_NOMEM;
         goto done;
     }
@@ -335,6 +388,14 @@ int oref_swattn_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, dou
                     xv[tok * d + c] = bf16_to_f64(v[src + c]);
                 }
             }
+            /* the extra segment of this (b, head), widened to fp64 */
+            for (tok = 0; tok < E; ++tok) {
+                long src = (((long)b * E + tok) * heads + hd) * d;
+                for (c = 0; c < d; ++c) {
+                    xkx[tok * d + c] = bf16_to_f64(kxb[src + c]);
+                    xvx[tok * d + c] = bf16_to_f64(vxb[src + c]);
+                }
+            }
             /* stage 1: roll by -Delta */
             roll_grid(xq, rq, &g, d, -1);
             roll_grid(xk, rk, &g, d, -1);
@@ -346,6 +407,7 @@ int oref_swattn_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, dou
             /* stage 3: attention in every window */
             job.g = &g; job.qw = wq; job.kw = wk; job.vw = wv; job.ow = wo;
             job.count = count; job.d = d; job.scale = scale; job.next = 0; job.failed = 0;
+            job.kx = xkx; job.vx = xvx; job.E = E;
             tids = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nthreads);
             if (!tids) { rc = OREF_ERR_NOMEM; goto done; }
             for (i = 0; i < nthreads; ++i)
@@ -368,8 +430,33 @@ int oref_swattn_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, dou
     }
 done:
     free(xq); free(xk); free(xv); free(rq); free(rk); free(rv); free(ro); free(y);
-    free(wq); free(wk); free(wv); free(wo); free(count);
+    free(wq); free(wk); free(wv); free(wo); free(count); free(xkx); free(xvx);
     return rc;
+}
+
+int oref_swattn_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, double *out,
+                    int B, int heads, int T, int H, int W, int d,
+                    const int win[3], const int shift[3], double scale,
+                    int head_begin, int head_end, int nthreads)
+{
+    return swattn_fwd_impl(q, k, v, NULL, NULL, 0, out, B, heads, T, H, W, d, win, shift, scale,
+                           head_begin, head_end, nthreads);
+}
+
+/*
+ * The forward with an extra key/value segment appended to every window
+ * (§3.2): kx, vx are bf16 [B, E, heads, d]; every query of window m attends
+ * to the window's tokens and to the E extra tokens of its own (b, head).
+ */
+int oref_swattn_fwd_mem(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                        const uint16_t *kx, const uint16_t *vx, int E, double *out,
+                        int B, int heads, int T, int H, int W, int d,
+                        const int win[3], const int shift[3], double scale,
+                        int head_begin, int head_end, int nthreads)
+{
+    if (E < 0 || (E > 0 && (!kx || !vx))) return OREF_ERR_ARG;
+    return swattn_fwd_impl(q, k, v, kx, vx, E, out, B, heads, T, H, W, d, win, shift, scale,
+                           head_begin, head_end, nthreads);
 }
 
 /* ------------------------------------------------------------------ */
@@ -484,4 +571,57 @@ double oref_flops(int B, int heads, int T, int H, int W, int d, const int win[3]
                 total += 4.0 * n * n * d;
             }
     return total * B * heads;
+}
+
+/* ------------------------------------------------------------------ */
+/* K/V pooling (§3.2 "K/V-Pooled Global Memory")                       */
+/* ------------------------------------------------------------------ */
+
+/*
+ * xbar[b, g, head, :] = the mean of x[b, token, head, :] over the tokens of
+ * patch g, where the original (unshifted) grid is cut into patches of
+ * p_t x p_h x p_w tokens, [g_a p_a, min((g_a + 1) p_a, n_a)) along each axis a
+ * (a truncated last patch averages over the tokens it has), and patches are
+ * numbered in raster order over (g_t, g_h, g_w).  x is bf16 [B, N, heads, d];
+ * xbar is fp64 [B, G, heads, d] with G = prod ceil(n_a / p_a).
+ */
+int oref_kv_pool(const uint16_t *x, double *xbar, int B, int heads, int T, int H, int W, int d,
+                 const int pool[3])
+{
+    const int n[3] = {T, H, W};
+    int G[3], a;
+    long g, Gt, N;
+    int b, hd, c;
+    if (!x || !xbar || !pool || B < 1 || heads < 1 || d < 1 || T < 1 || H < 1 || W < 1)
+        return OREF_ERR_ARG;
+    for (a = 0; a < 3; ++a) {
+        if (pool[a] < 1) return OREF_ERR_ARG;
+        G[a] = (n[a] + pool[a] - 1) / pool[a];
+    }
+    Gt = (long)G[0] * G[1] * G[2];
+    N = (long)T * H * W;
+    for (b = 0; b < B; ++b)
+        for (g = 0; g < Gt; ++g) {
+            const int gw = (int)(g % G[2]);
+            const int gh = (int)((g / G[2]) % G[1]);
+            const int gt = (int)(g / ((long)G[1] * G[2]));
+            const int t0 = gt * pool[0], h0 = gh * pool[1], w0 = gw * pool[2];
+            const int t1 = t0 + pool[0] < T ? t0 + pool[0] : T;
+            const int h1 = h0 + pool[1] < H ? h0 + pool[1] : H;
+            const int w1 = w0 + pool[2] < W ? w0 + pool[2] : W;
+            const double cnt = (double)(t1 - t0) * (h1 - h0) * (w1 - w0);
+            for (hd = 0; hd < heads; ++hd)
+                for (c = 0; c < d; ++c) {
+                    double acc = 0.0;
+                    int t, h, w;
+                    for (t = t0; t < t1; ++t)
+                        for (h = h0; h < h1; ++h)
+                            for (w = w0; w < w1; ++w) {
+                                const long tok = ((long)t * H + h) * W + w;
+                                acc += bf16_to_f64(x[(((long)b * N + tok) * heads + hd) * d + c]);
+                            }
+                    xbar[(((long)b * Gt + g) * heads + hd) * d + c] = acc / cnt;
+                }
+        }
+    return OREF_OK;
 }

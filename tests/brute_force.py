@@ -56,3 +56,40 @@ def masked_window_attention(q, k, v, T, H, W, win, shift, scale):
     wid = window_id_of_token(T, H, W, win, shift)
     mask = wid[:, None] == wid[None, :]
     return full_attention(q, k, v, scale, mask)
+
+
+def pooled_means(x, T, H, W, pool):
+    """[B, G, heads, d] patch means of x (fp64 [B, N, heads, d]) over the unshifted grid,
+    built with explicit numpy slicing of each patch (§3.2 "K/V-Pooled Global Memory")."""
+    B, N, heads, d = x.shape
+    g = x.reshape(B, T, H, W, heads, d)
+    out = []
+    for t0 in range(0, T, pool[0]):
+        for h0 in range(0, H, pool[1]):
+            for w0 in range(0, W, pool[2]):
+                patch = g[:, t0:t0 + pool[0], h0:h0 + pool[1], w0:w0 + pool[2]]
+                out.append(patch.reshape(B, -1, heads, d).mean(axis=1))
+    return np.stack(out, axis=1)
+
+
+def masked_window_attention_with_extra(q, k, v, kx, vx, T, H, W, win, shift, scale):
+    """Shifted-window attention where every query may also attend to the extra
+    tokens kx, vx ([B, E, heads, d]): full attention over the concatenated key set
+    [K; K_x] with the block-diagonal window mask widened by E always-allowed columns."""
+    E = kx.shape[1]
+    wid = window_id_of_token(T, H, W, win, shift)
+    mask = np.concatenate([wid[:, None] == wid[None, :],
+                           np.ones((wid.size, E), dtype=bool)], axis=1)
+    kk = np.concatenate([k, kx], axis=1)
+    vv = np.concatenate([v, vx], axis=1)
+    B, N, heads, d = q.shape
+    out = np.empty_like(q)
+    for b in range(B):
+        for h in range(heads):
+            s = scale * (q[b, :, h, :] @ kk[b, :, h, :].T)
+            s = np.where(mask, s, -np.inf)
+            s = s - s.max(axis=1, keepdims=True)
+            p = np.exp(s)
+            p /= p.sum(axis=1, keepdims=True)
+            out[b, :, h, :] = p @ vv[b, :, h, :]
+    return out

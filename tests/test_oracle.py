@@ -298,3 +298,72 @@ def test_shift_schedule_rejects_bad_arguments():
         oracle.shift_schedule(0, (1, 8, 8))
     with pytest.raises(ValueError):
         oracle.shift_schedule(4, (1, 0, 8))
+
+
+# ---------------------------------------------------------------- pooled global memory (§3.2)
+
+@pytest.mark.parametrize("grid,pool", [
+    ((1, 8, 8), (1, 4, 4)),
+    ((2, 5, 7), (1, 2, 3)),          # truncated patches on h and w
+    ((3, 4, 6), (2, 4, 4)),          # temporal pooling, truncated along t and w
+])
+def test_kv_pool_matches_patch_means(grid, pool):
+    from brute_force import pooled_means
+    T, H, W = grid
+    bits, (q, k, v) = _qkv(2, 3, 8, T, H, W, seed=sum(grid))
+    got = oracle.kv_pool(bits[1], 2, 3, T, H, W, 8, pool)
+    ref = pooled_means(k, T, H, W, pool)
+    assert got.shape == ref.shape == (2, oracle.n_pooled(T, H, W, pool), 3, 8)
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-14)
+
+
+def test_kv_pool_special_cases():
+    T, H, W = 2, 3, 5
+    bits, (q, k, v) = _qkv(1, 2, 4, T, H, W, seed=3)
+    # patches of one token: the pooled tokens are the tokens themselves, in raster order
+    np.testing.assert_array_equal(oracle.kv_pool(bits[2], 1, 2, T, H, W, 4, (1, 1, 1)), v)
+    # one patch covering the grid: the mean over all tokens
+    np.testing.assert_allclose(oracle.kv_pool(bits[2], 1, 2, T, H, W, 4, (T, H, W))[:, 0],
+                               v.mean(axis=1), rtol=0, atol=1e-15)
+    # hand-worked: a 1x2x2 grid of one channel pooled 2x2 -> the mean of its four values
+    x = oracle.round_to_bf16_bits(np.array([1.0, 2.0, 4.0, 8.0]).reshape(1, 4, 1, 1))
+    assert oracle.kv_pool(x, 1, 1, 1, 2, 2, 1, (1, 2, 2))[0, 0, 0, 0] == 3.75
+
+
+@pytest.mark.parametrize("grid,win,shift,E", [
+    ((1, 8, 8), (1, 4, 4), (0, 2, 2), 5),
+    ((2, 5, 7), (1, 3, 4), (1, 4, 6), 9),        # 3D, truncated windows
+    ((1, 6, 6), (1, 6, 6), (0, 0, 0), 3),        # one window: full attention plus the extra keys
+])
+def test_fwd_with_extra_segment_matches_masked_attention(grid, win, shift, E):
+    from brute_force import masked_window_attention_with_extra
+    T, H, W = grid
+    B, heads, d = 2, 2, 8
+    bits, (q, k, v) = _qkv(B, heads, d, T, H, W, seed=E)
+    xbits, (kx, vx, _) = _qkv(B, heads, d, 1, 1, E, seed=100 + E)
+    scale = 0.6 / math.sqrt(d)
+    got = oracle.swattn_fwd_mem(*bits, xbits[0], xbits[1], E, B, heads, T, H, W, d, win, shift, scale)
+    ref = masked_window_attention_with_extra(q, k, v, kx, vx, T, H, W, win, shift, scale)
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+
+
+def test_fwd_with_empty_extra_segment_is_the_plain_forward():
+    T, H, W = 1, 6, 8
+    bits, _ = _qkv(1, 2, 8, T, H, W, seed=4)
+    empty = np.zeros(0, dtype=np.uint16)
+    a = oracle.swattn_fwd_mem(*bits, empty, empty, 0, 1, 2, T, H, W, 8, (1, 3, 4), (0, 1, 2), 0.3)
+    b = oracle.swattn_fwd(*bits, 1, 2, T, H, W, 8, (1, 3, 4), (0, 1, 2), 0.3)
+    np.testing.assert_array_equal(a, b)
+
+
+def test_fwd_with_extra_segment_of_one_dominant_key():
+    # an extra key whose logit dominates every window key turns every output row into its value
+    T, H, W, d = 1, 4, 4, 4
+    bits, (q, k, v) = _qkv(1, 1, d, T, H, W, seed=9, dist="uniform")
+    qf = np.ones((1, T * H * W, 1, d))
+    qb = oracle.round_to_bf16_bits(qf)
+    kx = oracle.round_to_bf16_bits(np.full((1, 1, 1, d), 64.0))
+    vx = oracle.round_to_bf16_bits(np.arange(d, dtype=np.float64).reshape(1, 1, 1, d))
+    out = oracle.swattn_fwd_mem(qb, bits[1], bits[2], kx, vx, 1, 1, 1, T, H, W, d,
+                                (1, 2, 2), (0, 1, 1), 1.0)
+    np.testing.assert_allclose(out[0, :, 0, :], np.tile(np.arange(d), (T * H * W, 1)), rtol=0, atol=1e-30)
