@@ -468,6 +468,30 @@ def run_native(args):
                 "ms_per_stack": ms_stack, "ms_per_layer": ms_stack / len(shifts),
                 "tflops": f_layer * len(shifts) / ms_stack / 1e9,
                 "step_offset": [0, 0, 0]}
+        # Pooled global memory (§3.2): pool K/V into G tokens per (b, head), then
+        # the windowed forward with those G tokens appended to every window.
+        if args.memory_pool:
+            pool = tuple(int(x) for x in args.memory_pool.split(","))
+            G = sw.kv_pool_tokens(wl.grid, pool)
+            kbar, vbar = sw.kv_pool(k, v, wl.grid, pool, stream=stream)
+
+            def pool_only():
+                sw.kv_pool(k, v, wl.grid, pool, stream=stream)
+
+            def fwd_mem():
+                sw.swattn_fwd_mem(q, k, v, kbar, vbar, wl.grid, wl.win, wl.shifts[1], wl.scale,
+                                  out=out, stream=stream)
+            time_launches(fwd_mem, 2, stream)
+            ms_mem = statistics.median(time_launches(fwd_mem, 10, stream))
+            time_launches(pool_only, 2, stream)
+            ms_pool = statistics.median(time_launches(pool_only, 10, stream))
+            f_mem = f_layer + 4.0 * wl.B * wl.heads * wl.d * wl.N * G
+            extras["memory"] = {
+                "pool_thw": list(pool), "pooled_tokens": G, "shift_thw": list(wl.shifts[1]),
+                "ms_pool": ms_pool, "ms_fwd": ms_mem, "flops_fwd": f_mem,
+                "tflops_fwd": f_mem / ms_mem / 1e9,
+                "pool_gbs": 2 * (wl.B * wl.N + wl.B * G) * wl.heads * wl.d * 2 / ms_pool / 1e6}
+            del kbar, vbar
         # CPU baseline: the oracle on a bounded sample of the same workload
         if not args.no_cpu_baseline:
             qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
@@ -520,6 +544,8 @@ def main():
     ap.add_argument("--no-sweep", action="store_true", help="skip the per-workload table")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end timing")
+    ap.add_argument("--memory-pool", default="1,4,4",
+                    help="also time the pooled global memory: pooling factors t,h,w ('' to skip)")
     ap.add_argument("--schedule-layers", type=int, default=8,
                     help="also time an L-layer stack under the interleaved shift schedule (0: off)")
     ap.add_argument("--workload", default=HEADLINE,

@@ -93,6 +93,39 @@ int basa_swattn_flops(int B, int heads, int T, int H, int W, int d, const int wi
                       double* flops);
 
 /*
+ * The forward with an extra key/value segment (§3.2 "K/V-Pooled Global
+ * Memory": each window's keys and values become [K_W; K_bar], [V_W; V_bar]).
+ * kx, vx: device bf16 [B, E, heads, d], contiguous, 16-byte aligned: E extra
+ * tokens per (batch item, head), appended to the keys and values of every
+ * window of that (batch item, head) -- the pooled memory from basa_kv_pool,
+ * any other shared tokens (e.g. text), or both concatenated.  Queries and the
+ * output are unchanged: out[b, token, head, :] is the softmax attention of the
+ * query over its window's tokens and the E extra tokens.  E = 0 (kx, vx may
+ * then be null) is exactly basa_swattn_fwd.  Other arguments, errors and
+ * ownership as basa_swattn_fwd; out must not overlap kx or vx either.
+ */
+int basa_swattn_fwd_mem(const void* q, const void* k, const void* v, const void* kx,
+                        const void* vx, int E, void* out, int B, int heads, int T, int H, int W,
+                        int d, const int win[3], const int shift[3], float scale, void* stream);
+
+/*
+ * Pooled global memory (§3.2): kbar[b, g, head, :] and vbar[b, g, head, :]
+ * are the means of k and v over patch g of the unshifted grid.  The grid is cut
+ * into patches of pool[0] x pool[1] x pool[2] tokens (t, h, w), the last patch
+ * along an axis holding what is left; patches are numbered in raster order over
+ * (g_t, g_h, g_w), G = prod ceil(n_a / pool[a]) (basa_kv_pool_tokens).
+ * k, v: device bf16 [B, T*H*W, heads, d]; kbar, vbar: device bf16
+ * [B, G, heads, d] (fp32 sums, rounded to nearest even); all 16-byte aligned,
+ * outputs overlapping neither the inputs nor each other (BASA_ERR_ALIAS).
+ * d must be 64 or 128.  Asynchronous on `stream`.
+ */
+int basa_kv_pool(const void* k, const void* v, void* kbar, void* vbar, int B, int heads, int T,
+                 int H, int W, int d, const int pool[3], void* stream);
+
+/* Pooled tokens G = prod ceil(n_a / pool[a]) of a T x H x W grid, written to *G. */
+int basa_kv_pool_tokens(int T, int H, int W, const int pool[3], int* G);
+
+/*
  * The per-layer window offsets of the interleaved shift schedule
  * (§3.1 "Interleaved shift schedule"), per axis a with window w = win[a]:
  *   delta = max(1, floor(w / L)),  a_i = (i * delta) mod w  for i = 0..L-1,

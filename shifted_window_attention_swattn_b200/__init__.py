@@ -16,7 +16,8 @@ import os
 import threading
 
 __all__ = [
-    "swattn_fwd", "swattn_fwd_from_host", "index_map", "index_map_host", "flops", "shift_schedule",
+    "swattn_fwd", "swattn_fwd_from_host", "swattn_fwd_mem", "kv_pool", "kv_pool_tokens",
+    "index_map", "index_map_host", "flops", "shift_schedule",
     "last_device_error", "set_wait_timeout_ns", "strerror", "library_path", "SwattnError",
 ]
 
@@ -65,6 +66,12 @@ def _load():
         lib.basa_swattn_index_map_host.restype = ci
         lib.basa_swattn_flops.argtypes = [ci] * 6 + [_I3, ctypes.POINTER(ctypes.c_double)]
         lib.basa_swattn_flops.restype = ci
+        lib.basa_swattn_fwd_mem.argtypes = [vp] * 5 + [ci, vp] + [ci] * 6 + [_I3, _I3, ctypes.c_float, vp]
+        lib.basa_swattn_fwd_mem.restype = ci
+        lib.basa_kv_pool.argtypes = [vp] * 4 + [ci] * 6 + [_I3, vp]
+        lib.basa_kv_pool.restype = ci
+        lib.basa_kv_pool_tokens.argtypes = [ci, ci, ci, _I3, ctypes.POINTER(ctypes.c_int)]
+        lib.basa_kv_pool_tokens.restype = ci
         lib.basa_shift_schedule.argtypes = [ci, _I3, _I3, vp]
         lib.basa_shift_schedule.restype = ci
         lib.basa_swattn_last_device_error.argtypes = [vp]
@@ -130,6 +137,79 @@ def swattn_fwd(q, k, v, grid, win, shift, scale=None, out=None, stream=None):
     if rc != BASA_OK:
         raise SwattnError(rc, "basa_swattn_fwd")
     return out
+
+
+def swattn_fwd_mem(q, k, v, kx, vx, grid, win, shift, scale=None, out=None, stream=None):
+    """Shifted-window attention whose every window also attends to an extra K/V
+    segment (§3.2): kx, vx are bf16 CUDA tensors [B, E, heads, d] (pooled memory
+    from ``kv_pool``, other shared tokens, or both concatenated along dim 1)."""
+    import torch
+    lib = _load()
+    T, H, W = _triple(grid, "grid")
+    w3, s3 = _triple(win, "win"), _triple(shift, "shift")
+    for name, t in (("q", q), ("k", k), ("v", v), ("kx", kx), ("vx", vx)):
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or not t.is_cuda:
+            raise TypeError(f"{name} must be a bf16 CUDA tensor")
+        if not t.is_contiguous() or t.dim() != 4:
+            raise ValueError(f"{name} must be contiguous and 4-D")
+    if q.shape != k.shape or q.shape != v.shape:
+        raise ValueError("q, k, v must have the same shape")
+    B, N, heads, d = q.shape
+    if kx.shape != vx.shape or kx.shape[0] != B or kx.shape[2:] != q.shape[2:]:
+        raise ValueError("kx, vx must be [B, E, heads, d] like q")
+    if N != T * H * W:
+        raise ValueError(f"token count {N} != T*H*W = {T * H * W}")
+    if out is None:
+        out = torch.empty_like(q)
+    elif out.shape != q.shape or out.dtype != torch.bfloat16 or not out.is_contiguous():
+        raise ValueError("out must be a contiguous bf16 tensor shaped like q")
+    if scale is None:
+        scale = d ** -0.5
+    E = kx.shape[1]
+    rc = lib.basa_swattn_fwd_mem(q.data_ptr(), k.data_ptr(), v.data_ptr(), kx.data_ptr(), vx.data_ptr(),
+                                 E, out.data_ptr(), B, heads, T, H, W, d, _I3(*w3), _I3(*s3),
+                                 float(scale), _stream_handle(stream, q.device))
+    if rc != BASA_OK:
+        raise SwattnError(rc, "basa_swattn_fwd_mem")
+    return out
+
+
+def kv_pool_tokens(grid, pool) -> int:
+    """Pooled tokens G = prod ceil(n_a / pool_a) (§3.2)."""
+    lib = _load()
+    T, H, W = _triple(grid, "grid")
+    G = ctypes.c_int(0)
+    rc = lib.basa_kv_pool_tokens(T, H, W, _I3(*_triple(pool, "pool")), ctypes.byref(G))
+    if rc != BASA_OK:
+        raise SwattnError(rc, "basa_kv_pool_tokens")
+    return G.value
+
+
+def kv_pool(k, v, grid, pool, stream=None):
+    """Pooled global memory (§3.2): (kbar, vbar), bf16 [B, G, heads, d] patch means of
+    k and v over the unshifted grid, patches of pool = (p_t, p_h, p_w) in raster order."""
+    import torch
+    lib = _load()
+    T, H, W = _triple(grid, "grid")
+    p3 = _triple(pool, "pool")
+    for name, t in (("k", k), ("v", v)):
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or not t.is_cuda:
+            raise TypeError(f"{name} must be a bf16 CUDA tensor")
+        if not t.is_contiguous() or t.dim() != 4:
+            raise ValueError(f"{name} must be contiguous [B, T*H*W, heads, d]")
+    if k.shape != v.shape:
+        raise ValueError("k and v must have the same shape")
+    B, N, heads, d = k.shape
+    if N != T * H * W:
+        raise ValueError(f"token count {N} != T*H*W = {T * H * W}")
+    G = kv_pool_tokens(grid, p3)
+    kbar = torch.empty((B, G, heads, d), dtype=torch.bfloat16, device=k.device)
+    vbar = torch.empty_like(kbar)
+    rc = lib.basa_kv_pool(k.data_ptr(), v.data_ptr(), kbar.data_ptr(), vbar.data_ptr(), B, heads,
+                          T, H, W, d, _I3(*p3), _stream_handle(stream, k.device))
+    if rc != BASA_OK:
+        raise SwattnError(rc, "basa_kv_pool")
+    return kbar, vbar
 
 
 def swattn_fwd_from_host(q_host, k_host, v_host, grid, win, shift, scale=None, out_host=None,

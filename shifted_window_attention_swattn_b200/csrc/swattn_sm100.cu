@@ -141,6 +141,8 @@ static int make_geometry(Geometry* g, int T, int H, int W, const int win[3], con
 
 struct __align__(64) FwdParams {
   CUtensorMap tq, tk, tv;       // 2D [rows = B*N*heads, cols = d], box {64, 1}, 128B swizzle
+  CUtensorMap tkx, tvx;         // extra K/V segment, 2D [rows = B*n_extra*heads, cols = d] (kMem)
+  int n_extra;                  // extra keys appended to every window (kMem)
   __nv_bfloat16* out;
   Geometry g;
   int B, heads, d;
@@ -195,12 +197,15 @@ struct Unit {
   int m[3], e[3];
   int n_valid;    // tokens in the window
   int q0;         // first query slot of tile 0
-  int nkv;        // key tiles
+  int nkv;        // key tiles: the window's, then (kMem) those of the extra segment
+  int nkv_win;    // key tiles of the window
+  int n_extra;    // keys of the extra segment (kMem), else 0
   bool has_q1;    // tile 1 holds at least one query
 };
 
 // Units are numbered with the query pair fastest, then window, then
 // (batch, head), so CTAs that run at the same time share K/V in L2.
+template <bool kMem>
 __device__ __forceinline__ bool decode_unit(const FwdParams& p, int u, Unit& U) {
   const int qp = u % p.q_pairs;
   const int r = u / p.q_pairs;
@@ -214,6 +219,9 @@ __device__ __forceinline__ bool decode_unit(const FwdParams& p, int u, Unit& U) 
   if (U.q0 >= U.n_valid) return false;   // a truncated window has fewer query pairs
   U.has_q1 = U.q0 + kTile < U.n_valid;
   U.nkv = (U.n_valid + kTile - 1) / kTile;
+  U.nkv_win = U.nkv;
+  U.n_extra = kMem ? p.n_extra : 0;
+  if (kMem) U.nkv += (p.n_extra + kTile - 1) / kTile;
   return true;
 }
 
@@ -222,9 +230,26 @@ __device__ __forceinline__ int unit_row(const FwdParams& p, const Unit& U, int s
   return (U.b * p.g.N + slot_token(p.g, U.m, U.e, slot)) * p.heads + U.h;
 }
 
+// Valid keys of key tile j: the window's tiles, then (kMem) the extra segment's.
+template <bool kMem>
 __device__ __forceinline__ int kv_valid_of(const Unit& U, int j) {
+  if (kMem && j >= U.nkv_win) {
+    const int left = U.n_extra - (j - U.nkv_win) * kTile;
+    return left < kTile ? left : kTile;
+  }
   const int left = U.n_valid - j * kTile;
   return left < kTile ? left : kTile;
+}
+
+// Rows of the extra segment's tokens s .. s+3 for unit U in the 2D
+// [B*n_extra*heads, d] view of the extra K/V: row = (b*n_extra + token)*heads + h;
+// tokens at or past n_extra repeat the last one.
+__device__ __forceinline__ void extra_rows4(const Unit& U, int heads, int s, int r[4]) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int t = s + k < U.n_extra ? s + k : U.n_extra - 1;
+    r[k] = (U.b * U.n_extra + t) * heads + U.h;
+  }
 }
 
 // Rows of slots s .. s+3 of unit U in the 2D [B*N*heads, d] view of Q/K/V/out,
@@ -326,6 +351,7 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint3
             (accumulate || kk > 0) ? 1u : 0u);
 }
 
+template <bool kMem>
 __global__ void __launch_bounds__(kThreads, 1) swattn_fwd_kernel(const __grid_constant__ FwdParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -383,20 +409,25 @@ __global__ void __launch_bounds__(kThreads, 1) swattn_fwd_kernel(const __grid_co
     uint32_t q_use[2] = {0, 0};
     uint32_t ld = 0;          // loads issued into the ring
     bool ok = true;
-    auto issue = [&](const Unit& U, int slot0, const CUtensorMap* map, uint64_t* bar, uint8_t* tile) {
+    // extra: the tile comes from the extra K/V segment (slot0 counts its tokens).
+    auto issue = [&](const Unit& U, int slot0, const CUtensorMap* map, uint64_t* bar, uint8_t* tile,
+                     bool extra) {
       if (elect_one()) mbar_arrive_expect_tx(bar, half_bytes);
       __syncwarp();
       for (int n = pw + kProducers * lane; n < 32 * ncb; n += 32 * kProducers) {
         const int grp = n / ncb, c = n - grp * ncb;
         int r[4];
-        unit_rows4(p.g, U, p.heads, slot0 + 4 * grp, r);
+        if (kMem && extra)
+          extra_rows4(U, p.heads, slot0 + 4 * grp, r);
+        else
+          unit_rows4(p.g, U, p.heads, slot0 + 4 * grp, r);
         tma_gather4(map, bar, tile + c * (kTile * 128) + grp * 512, c * 64, r[0], r[1], r[2], r[3]);
       }
       __syncwarp();
     };
     for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
       Unit U;
-      if (!decode_unit(p, u, U)) continue;
+      if (!decode_unit<kMem>(p, u, U)) continue;
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
         if (i == 1 && !U.has_q1) break;
@@ -405,7 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1) swattn_fwd_kernel(const __grid_co
                           wait_or_abort(&ctl->q_empty[i], (q_use[i] - 1) & 1, ctl, p.timeout_ns));
           if (!ok) break;
         }
-        issue(U, U.q0 + i * kTile, &p.tq, &ctl->q_full[i], sQ + i * tile_bytes);
+        issue(U, U.q0 + i * kTile, &p.tq, &ctl->q_full[i], sQ + i * tile_bytes, false);
         ++q_use[i];
       }
       for (int j = 0; ok && j < U.nkv; ++j) {
@@ -417,7 +448,12 @@ __global__ void __launch_bounds__(kThreads, 1) swattn_fwd_kernel(const __grid_co
                             wait_or_abort(&ctl->kv_empty[slot], (use - 1) & 1, ctl, p.timeout_ns));
             if (!ok) break;
           }
-          issue(U, j * kTile, kv == 0 ? &p.tk : &p.tv, &ctl->kv_full[slot], sRing + slot * tile_bytes);
+          if (kMem && j >= U.nkv_win)
+            issue(U, (j - U.nkv_win) * kTile, kv == 0 ? &p.tkx : &p.tvx, &ctl->kv_full[slot],
+                  sRing + slot * tile_bytes, true);
+          else
+            issue(U, j * kTile, kv == 0 ? &p.tk : &p.tv, &ctl->kv_full[slot], sRing + slot * tile_bytes,
+                  false);
           ++ld;
         }
       }
@@ -441,7 +477,7 @@ __global__ void __launch_bounds__(kThreads, 1) swattn_fwd_kernel(const __grid_co
       bool ok = !p.stall || wait_or_abort(&ctl->never, 0, ctl, p.timeout_ns);
       for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
         Unit U;
-        if (!decode_unit(p, u, U)) continue;
+        if (!decode_unit<kMem>(p, u, U)) continue;
         const int nq = U.has_q1 ? 2 : 1;
 #pragma unroll
         for (int i = 0; i < 2; ++i)
@@ -454,7 +490,7 @@ __global__ void __launch_bounds__(kThreads, 1) swattn_fwd_kernel(const __grid_co
         ++ld;
         tc_fence_after();
         {
-          const int n_s = (kv_valid_of(U, 0) + 15) & ~15;
+          const int n_s = (kv_valid_of<kMem>(U, 0) + 15) & ~15;
 #pragma unroll
           for (int i = 0; i < 2; ++i) {
             if (i >= nq) break;
@@ -470,7 +506,7 @@ __global__ void __launch_bounds__(kThreads, 1) swattn_fwd_kernel(const __grid_co
           if (!ok) break;
           ++ld;
           const bool more = j + 1 < U.nkv;
-          const int kvv = kv_valid_of(U, j);
+          const int kvv = kv_valid_of<kMem>(U, j);
 #pragma unroll
           for (int i = 0; i < 2; ++i) {
             if (i >= nq) break;
@@ -489,7 +525,7 @@ __global__ void __launch_bounds__(kThreads, 1) swattn_fwd_kernel(const __grid_co
                 ++ld;
                 tc_fence_after();
               }
-              const int n_s = (kv_valid_of(U, j + 1) + 15) & ~15;
+              const int n_s = (kv_valid_of<kMem>(U, j + 1) + 15) & ~15;
               issue_qk(tS[i], q_addr[i], ring_addr + slot_k * tile_bytes, d, n_s);
               umma_commit(&ctl->s_full[i]);
               if (j + 1 == U.nkv - 1) umma_commit(&ctl->q_empty[i]);
@@ -518,7 +554,7 @@ __global__ void __launch_bounds__(kThreads, 1) swattn_fwd_kernel(const __grid_co
     bool ok = true;
     for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
       Unit U;
-      if (!decode_unit(p, u, U)) continue;
+      if (!decode_unit<kMem>(p, u, U)) continue;
       if (wg == 1 && !U.has_q1) continue;
       float m_run = -INFINITY;   // running max of scale*log2(e)*S (possibly stale by < 8)
       float l_run = 0.0f;        // running sum of exp2(x - m_run)
@@ -529,7 +565,7 @@ __global__ void __launch_bounds__(kThreads, 1) swattn_fwd_kernel(const __grid_co
         tc_fence_after();
         float alpha;
         bool need;
-        const float rowsum = softmax_row_step(tS, kv_valid_of(U, j), sl2, m_run, alpha, need);
+        const float rowsum = softmax_row_step(tS, kv_valid_of<kMem>(U, j), sl2, m_run, alpha, need);
         l_run = l_run * alpha + rowsum;
         if (j > 0 && __any_sync(0xffffffffu, need)) {
           // O_i holds P V of tiles 0..j-1 (complete: S_i(j) was issued after
@@ -614,6 +650,8 @@ constexpr int kPairMaxSlots = 12;
 
 struct __align__(64) PairParams {
   CUtensorMap tq, tk, tv;       // 2D [rows = B*N*heads, cols = 128], box {64, 1}, 128B swizzle
+  CUtensorMap tkx, tvx;         // extra K/V segment, 2D [rows = B*n_extra*heads, cols = 128] (kMem)
+  int n_extra;                  // extra keys appended to every window (kMem)
   __nv_bfloat16* out;
   Geometry g;
   int B, heads;
@@ -653,6 +691,7 @@ __device__ __forceinline__ bool pair_wait(uint64_t* bar, uint32_t parity, PairCt
 }
 
 // A pair unit: up to 512 queries; tile i of CTA c holds slots q0 + 256 i + 128 c + [0, 128).
+template <bool kMem>
 __device__ __forceinline__ bool decode_pair_unit(const PairParams& p, int u, Unit& U) {
   const int qp = u % p.q_quads;
   const int r = u / p.q_quads;
@@ -666,6 +705,9 @@ __device__ __forceinline__ bool decode_pair_unit(const PairParams& p, int u, Uni
   if (U.q0 >= U.n_valid) return false;
   U.has_q1 = U.q0 + 2 * kTile < U.n_valid;
   U.nkv = (U.n_valid + kTile - 1) / kTile;
+  U.nkv_win = U.nkv;
+  U.n_extra = kMem ? p.n_extra : 0;
+  if (kMem) U.nkv += (p.n_extra + kTile - 1) / kTile;
   return true;
 }
 
@@ -676,11 +718,13 @@ __device__ __forceinline__ int pair_row(const PairParams& p, const Unit& U, int 
 
 // Keys of tile j used by the MMAs: all 128, or the valid keys rounded up to 32
 // for the last tile (each CTA then holds half of them).
+template <bool kMem>
 __device__ __forceinline__ int pair_ns(const Unit& U, int j) {
-  const int kvv = kv_valid_of(U, j);
+  const int kvv = kv_valid_of<kMem>(U, j);
   return kvv == kTile ? kTile : ((kvv + 31) & ~31);
 }
 
+template <bool kMem>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     swattn_fwd_pair_kernel(const __grid_constant__ PairParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -745,14 +789,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     // producer warp n mod P (P producer warps), which computes its own four row
     // coordinates; every lane with a gather issues it in the same instruction, so
     // a warp puts up to 32 gathers in flight per issue.
+    // extra: the rows come from the extra K/V segment (slot0 counts its tokens).
     auto gathers = [&](const Unit& U, const CUtensorMap* map, uint32_t bar_leader, uint8_t* dst,
-                       int slot0, int count, int nblk, int blk_stride, int col0) {
+                       int slot0, int count, int nblk, int blk_stride, int col0, bool extra) {
       for (int base = 0; base < count; base += 32 * kPairProducers) {
         const int n = base + pw + kPairProducers * lane;
         if (n < count) {
           const int grp = n / nblk, blk = n - grp * nblk;
           int r[4];
-          unit_rows4(p.g, U, p.heads, slot0 + 4 * grp, r);
+          if (kMem && extra)
+            extra_rows4(U, p.heads, slot0 + 4 * grp, r);
+          else
+            unit_rows4(p.g, U, p.heads, slot0 + 4 * grp, r);
           tma_gather4_pair(map, bar_leader, dst + grp * 512 + blk * blk_stride, col0 + 64 * blk, r[0],
                            r[1], r[2], r[3]);
         }
@@ -761,7 +809,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     };
     for (int u = cluster_id; ok && u < p.total_units; u += n_clusters) {
       Unit U;
-      if (!decode_pair_unit(p, u, U)) continue;
+      if (!decode_pair_unit<kMem>(p, u, U)) continue;
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
         if (i == 1 && !U.has_q1) break;
@@ -774,11 +822,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         if (leader && pw == 0 && elect_one()) mbar_arrive_expect_tx(&ctl->q_full[i], 2 * kQBytes);
         __syncwarp();
         gathers(U, &p.tq, bar, sQ + i * kQBytes, U.q0 + i * 2 * kTile + static_cast<int>(rank) * kTile, 64, 2,
-                kTile * 128, 0);
+                kTile * 128, 0, false);
         ++q_use[i];
       }
       for (int j = 0; ok && j < U.nkv; ++j) {
-        const int ns = pair_ns(U, j);
+        const int ns = pair_ns<kMem>(U, j);
         const int half = ns >> 1;
         for (int kv = 0; kv < 2; ++kv) {
           const int slot = ld % n_slots;
@@ -793,10 +841,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             mbar_arrive_expect_tx(&ctl->kv_full[slot], static_cast<uint32_t>(ns) * 256u);
           __syncwarp();
           uint8_t* dst = sRing + slot * kPairHalfTileBytes;
+          // Tiles past the window's come from the extra segment (kMem).
+          const bool extra = kMem && j >= U.nkv_win;
+          const int t0 = extra ? (j - U.nkv_win) * kTile : j * kTile;
           if (kv == 0)   // K: keys [rank*half, rank*half + half), both column blocks
-            gathers(U, &p.tk, bar, dst, j * kTile + static_cast<int>(rank) * half, (half >> 2) * 2, 2, 64 * 128, 0);
+            gathers(U, extra ? &p.tkx : &p.tk, bar, dst, t0 + static_cast<int>(rank) * half, (half >> 2) * 2, 2,
+                    64 * 128, 0, extra);
           else           // V: keys [0, ns), the column block of this CTA's half of d
-            gathers(U, &p.tv, bar, dst, j * kTile, ns >> 2, 1, 0, 64 * static_cast<int>(rank));
+            gathers(U, extra ? &p.tvx : &p.tv, bar, dst, t0, ns >> 2, 1, 0, 64 * static_cast<int>(rank), extra);
           ++ld;
         }
       }
@@ -838,7 +890,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       };
       for (int u = cluster_id; ok && u < p.total_units; u += n_clusters) {
         Unit U;
-        if (!decode_pair_unit(p, u, U)) continue;
+        if (!decode_pair_unit<kMem>(p, u, U)) continue;
         const int nq = U.has_q1 ? 2 : 1;
 #pragma unroll
         for (int i = 0; i < 2; ++i)
@@ -852,7 +904,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
           if (i >= nq) break;
-          issue_qk(i, ring_addr + slot_k * kPairHalfTileBytes, pair_ns(U, 0));
+          issue_qk(i, ring_addr + slot_k * kPairHalfTileBytes, pair_ns<kMem>(U, 0));
           umma_commit_pair(&ctl->s_full[i], 3);
           if (U.nkv == 1) umma_commit_pair(&ctl->q_empty[i], 3);
         }
@@ -863,7 +915,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           if (!ok) break;
           ++ld;
           const bool more = j + 1 < U.nkv;
-          const int ns = pair_ns(U, j);
+          const int ns = pair_ns<kMem>(U, j);
 #pragma unroll
           for (int i = 0; i < 2; ++i) {
             if (i >= nq) break;
@@ -882,7 +934,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                 ++ld;
                 tc_fence_after();
               }
-              issue_qk(i, ring_addr + slot_k * kPairHalfTileBytes, pair_ns(U, j + 1));
+              issue_qk(i, ring_addr + slot_k * kPairHalfTileBytes, pair_ns<kMem>(U, j + 1));
               umma_commit_pair(&ctl->s_full[i], 3);
               if (j + 1 == U.nkv - 1) umma_commit_pair(&ctl->q_empty[i], 3);
               if (i == nq - 1) umma_commit_pair(&ctl->kv_empty[slot_k], 3);
@@ -910,7 +962,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     bool ok = true;
     for (int u = cluster_id; ok && u < p.total_units; u += n_clusters) {
       Unit U;
-      if (!decode_pair_unit(p, u, U)) continue;
+      if (!decode_pair_unit<kMem>(p, u, U)) continue;
       if (wg == 1 && !U.has_q1) continue;
       float m_run = -INFINITY;
       float l_run = 0.0f;
@@ -921,7 +973,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         tc_fence_after();
         float alpha;
         bool need;
-        const float rowsum = softmax_row_step(tS, kv_valid_of(U, j), sl2, m_run, alpha, need);
+        const float rowsum = softmax_row_step(tS, kv_valid_of<kMem>(U, j), sl2, m_run, alpha, need);
         l_run = l_run * alpha + rowsum;
         if (j > 0 && __any_sync(0xffffffffu, need)) {
           for (int c = 0; c < 4; ++c) {
@@ -972,6 +1024,64 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   if (warp == kPairMmaWarp) {
     tc_fence_after();
     tmem_dealloc_pair(tmem, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------ pooled global memory
+
+// §3.2 "K/V-Pooled Global Memory": xbar[b, g, head, :] = the mean of
+// x[b, token, head, :] over the tokens of patch g.  The unshifted grid is cut
+// into patches of pool[0] x pool[1] x pool[2] tokens (a truncated last patch
+// averages over the tokens it has), numbered in raster order over (g_t, g_h,
+// g_w).  One thread per (b, g, head, 8 channels): it sums its 16-byte slice of
+// every token row of the patch in fp32 and stores the mean as bf16 (RNE).
+// Consecutive threads read consecutive 16-byte pieces of a token row.
+struct PoolParams {
+  const __nv_bfloat16* x;
+  __nv_bfloat16* xbar;
+  int B, heads, d, T, H, W;
+  int pool[3], G[3];
+  long long total;   // B * G * heads * d / 8
+};
+
+__global__ void kv_pool_kernel(const PoolParams p) {
+  const int chunks = p.d / 8;
+  const long long Gt = static_cast<long long>(p.G[0]) * p.G[1] * p.G[2];
+  const long long N = static_cast<long long>(p.T) * p.H * p.W;
+  for (long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; idx < p.total;
+       idx += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int c = static_cast<int>(idx % chunks);
+    long long r = idx / chunks;
+    const int hd = static_cast<int>(r % p.heads);
+    r /= p.heads;
+    const long long g = r % Gt;
+    const int b = static_cast<int>(r / Gt);
+    const int gw = static_cast<int>(g % p.G[2]);
+    const int gh = static_cast<int>((g / p.G[2]) % p.G[1]);
+    const int gt = static_cast<int>(g / (static_cast<long long>(p.G[1]) * p.G[2]));
+    const int t0 = gt * p.pool[0], h0 = gh * p.pool[1], w0 = gw * p.pool[2];
+    const int t1 = min(t0 + p.pool[0], p.T), h1 = min(h0 + p.pool[1], p.H), w1 = min(w0 + p.pool[2], p.W);
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+    for (int t = t0; t < t1; ++t)
+      for (int h = h0; h < h1; ++h)
+        for (int w = w0; w < w1; ++w) {
+          const long long tok = (static_cast<long long>(t) * p.H + h) * p.W + w;
+          const uint4 v = *reinterpret_cast<const uint4*>(p.x + ((b * N + tok) * p.heads + hd) * p.d + c * 8);
+          const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            acc[2 * i] += __uint_as_float(u[i] << 16);
+            acc[2 * i + 1] += __uint_as_float(u[i] & 0xffff0000u);
+          }
+        }
+    const float inv = 1.0f / static_cast<float>((t1 - t0) * (h1 - h0) * (w1 - w0));
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) o[i] = pack_bf16x2(acc[2 * i] * inv, acc[2 * i + 1] * inv);
+    *reinterpret_cast<uint4*>(p.xbar + ((b * Gt + g) * p.heads + hd) * p.d + c * 8) =
+        make_uint4(o[0], o[1], o[2], o[3]);
   }
 }
 
@@ -1051,13 +1161,17 @@ static int prepare_device(int* dev_out) {
     g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
   }
   size_t smem_max = smem_bytes_for(128) > smem_bytes_for(64) ? smem_bytes_for(128) : smem_bytes_for(64);
-  if (cudaFuncSetAttribute(swattn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(swattn_fwd_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem_max)) != cudaSuccess ||
+      cudaFuncSetAttribute(swattn_fwd_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem_max)) != cudaSuccess)
     return BASA_ERR_CUDA;
   if (cudaDeviceGetAttribute(&g_sm_count[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
       g_sm_count[dev] < 1)
     return BASA_ERR_CUDA;
-  if (cudaFuncSetAttribute(swattn_fwd_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(swattn_fwd_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(pair_smem_bytes())) != cudaSuccess ||
+      cudaFuncSetAttribute(swattn_fwd_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(pair_smem_bytes())) != cudaSuccess)
     return BASA_ERR_CUDA;
   {
@@ -1066,10 +1180,12 @@ static int prepare_device(int* dev_out) {
     cfg.gridDim = dim3(2 * g_sm_count[dev], 1, 1);
     cfg.blockDim = dim3(kPairThreads, 1, 1);
     cfg.dynamicSmemBytes = pair_smem_bytes();
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, swattn_fwd_pair_kernel, &cfg) != cudaSuccess || n < 1)
+    int n = 0, n_mem = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, swattn_fwd_pair_kernel<false>, &cfg) != cudaSuccess || n < 1 ||
+        cudaOccupancyMaxActiveClusters(&n_mem, swattn_fwd_pair_kernel<true>, &cfg) != cudaSuccess ||
+        n_mem < 1)
       return BASA_ERR_CUDA;
-    g_pair_clusters[dev] = n;
+    g_pair_clusters[dev] = n < n_mem ? n : n_mem;
   }
   g_dev_state[dev] = 1;
   return BASA_OK;
@@ -1092,15 +1208,24 @@ static bool overlaps(const void* a, const void* b, size_t bytes) {
   return x < y + bytes && y < x + bytes;
 }
 
+// [a, a + na) and [b, b + nb) share a byte.
+static bool overlaps2(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return na > 0 && nb > 0 && x < y + nb && y < x + na;
+}
+
 }  // namespace swattn
 
 using namespace swattn;
 
-extern "C" int basa_swattn_fwd(const void* q, const void* k, const void* v, void* out, int B,
-                               int heads, int T, int H, int W, int d, const int win[3],
-                               const int shift[3], float scale, void* stream) {
+// The forward with an optional extra K/V segment of E tokens per (b, head)
+// appended to every window (E = 0: the plain forward).
+static int launch_fwd(const void* q, const void* k, const void* v, const void* kx, const void* vx,
+                      int E, void* out, int B, int heads, int T, int H, int W, int d, const int win[3],
+                      const int shift[3], float scale, void* stream) {
   if (!q || !k || !v || !out) return BASA_ERR_INVALID_ARG;
-  if (B < 1 || heads < 1) return BASA_ERR_INVALID_ARG;
+  if (B < 1 || heads < 1 || E < 0) return BASA_ERR_INVALID_ARG;
+  if (E > 0 && (!kx || !vx)) return BASA_ERR_INVALID_ARG;
   if (!std::isfinite(scale)) return BASA_ERR_INVALID_ARG;
   if (scale < 0.0f) return BASA_ERR_UNSUPPORTED;
   Geometry g;
@@ -1108,12 +1233,16 @@ extern "C" int basa_swattn_fwd(const void* q, const void* k, const void* v, void
   if (rc) return rc;
   if (d != 64 && d != 128) return BASA_ERR_UNSUPPORTED;
   const long long rows = static_cast<long long>(B) * g.N * heads;
-  if (rows >= (1LL << 31)) return BASA_ERR_UNSUPPORTED;
-  const void* ptrs[4] = {q, k, v, out};
+  const long long xrows = static_cast<long long>(B) * E * heads;
+  if (rows >= (1LL << 31) || xrows >= (1LL << 31)) return BASA_ERR_UNSUPPORTED;
+  const void* ptrs[6] = {q, k, v, out, E > 0 ? kx : q, E > 0 ? vx : q};
   for (const void* ptr : ptrs)
     if (reinterpret_cast<uintptr_t>(ptr) & 15) return BASA_ERR_ALIGNMENT;
   const size_t bytes = static_cast<size_t>(rows) * d * 2;
+  const size_t xbytes = static_cast<size_t>(xrows) * d * 2;
   if (overlaps(out, q, bytes) || overlaps(out, k, bytes) || overlaps(out, v, bytes))
+    return BASA_ERR_ALIAS;
+  if (E > 0 && (overlaps2(out, bytes, kx, xbytes) || overlaps2(out, bytes, vx, xbytes)))
     return BASA_ERR_ALIAS;
   const long long q_pairs = (g.nw_max + 2 * kTile - 1) / (2 * kTile);
   const long long units = static_cast<long long>(B) * heads * g.n_windows * q_pairs;
@@ -1133,6 +1262,9 @@ extern "C" int basa_swattn_fwd(const void* q, const void* k, const void* v, void
     if (encode_rows(&pp.tq, q, rows, d) || encode_rows(&pp.tk, k, rows, d) ||
         encode_rows(&pp.tv, v, rows, d))
       return BASA_ERR_CUDA;
+    if (E > 0 && (encode_rows(&pp.tkx, kx, xrows, d) || encode_rows(&pp.tvx, vx, xrows, d)))
+      return BASA_ERR_CUDA;
+    pp.n_extra = E;
     pp.out = static_cast<__nv_bfloat16*>(out);
     pp.g = g;
     pp.B = B;
@@ -1144,8 +1276,12 @@ extern "C" int basa_swattn_fwd(const void* q, const void* k, const void* v, void
     pp.timeout_ns = g_timeout_ns;
     pp.stall = g_stall;
     const long long clusters = punits < g_pair_clusters[dev] ? punits : g_pair_clusters[dev];
-    swattn_fwd_pair_kernel<<<static_cast<unsigned>(2 * clusters), kPairThreads, pair_smem_bytes(),
-                             static_cast<cudaStream_t>(stream)>>>(pp);
+    if (E > 0)
+      swattn_fwd_pair_kernel<true><<<static_cast<unsigned>(2 * clusters), kPairThreads, pair_smem_bytes(),
+                                     static_cast<cudaStream_t>(stream)>>>(pp);
+    else
+      swattn_fwd_pair_kernel<false><<<static_cast<unsigned>(2 * clusters), kPairThreads, pair_smem_bytes(),
+                                      static_cast<cudaStream_t>(stream)>>>(pp);
     return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;
   }
 
@@ -1154,6 +1290,9 @@ extern "C" int basa_swattn_fwd(const void* q, const void* k, const void* v, void
   if (encode_rows(&p.tq, q, rows, d) || encode_rows(&p.tk, k, rows, d) ||
       encode_rows(&p.tv, v, rows, d))
     return BASA_ERR_CUDA;
+  if (E > 0 && (encode_rows(&p.tkx, kx, xrows, d) || encode_rows(&p.tvx, vx, xrows, d)))
+    return BASA_ERR_CUDA;
+  p.n_extra = E;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.g = g;
   p.B = B;
@@ -1167,9 +1306,26 @@ extern "C" int basa_swattn_fwd(const void* q, const void* k, const void* v, void
   p.stall = g_stall;
   // Persistent: one CTA per SM, each walking the units with a stride of the grid.
   const long long grid = units < g_sm_count[dev] ? units : g_sm_count[dev];
-  swattn_fwd_kernel<<<static_cast<unsigned>(grid), kThreads, smem_bytes_for(d),
-                      static_cast<cudaStream_t>(stream)>>>(p);
+  if (E > 0)
+    swattn_fwd_kernel<true><<<static_cast<unsigned>(grid), kThreads, smem_bytes_for(d),
+                              static_cast<cudaStream_t>(stream)>>>(p);
+  else
+    swattn_fwd_kernel<false><<<static_cast<unsigned>(grid), kThreads, smem_bytes_for(d),
+                               static_cast<cudaStream_t>(stream)>>>(p);
   return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;
+}
+
+extern "C" int basa_swattn_fwd(const void* q, const void* k, const void* v, void* out, int B,
+                               int heads, int T, int H, int W, int d, const int win[3],
+                               const int shift[3], float scale, void* stream) {
+  return launch_fwd(q, k, v, nullptr, nullptr, 0, out, B, heads, T, H, W, d, win, shift, scale, stream);
+}
+
+extern "C" int basa_swattn_fwd_mem(const void* q, const void* k, const void* v, const void* kx,
+                                   const void* vx, int E, void* out, int B, int heads, int T, int H,
+                                   int W, int d, const int win[3], const int shift[3], float scale,
+                                   void* stream) {
+  return launch_fwd(q, k, v, kx, vx, E, out, B, heads, T, H, W, d, win, shift, scale, stream);
 }
 
 extern "C" int basa_swattn_index_map(int T, int H, int W, const int win[3], const int shift[3],
@@ -1223,6 +1379,65 @@ extern "C" int basa_swattn_flops(int B, int heads, int T, int H, int W, int d, c
   }
   *flops = 4.0 * s2 * d * static_cast<double>(B) * heads;
   return BASA_OK;
+}
+
+extern "C" int basa_kv_pool_tokens(int T, int H, int W, const int pool[3], int* G) {
+  if (!pool || !G || T < 1 || H < 1 || W < 1) return BASA_ERR_INVALID_ARG;
+  const int n[3] = {T, H, W};
+  long long g = 1;
+  for (int a = 0; a < 3; ++a) {
+    if (pool[a] < 1) return BASA_ERR_INVALID_ARG;
+    g *= (n[a] + pool[a] - 1) / pool[a];
+  }
+  if (g >= (1LL << 31)) return BASA_ERR_UNSUPPORTED;
+  *G = static_cast<int>(g);
+  return BASA_OK;
+}
+
+extern "C" int basa_kv_pool(const void* k, const void* v, void* kbar, void* vbar, int B, int heads,
+                            int T, int H, int W, int d, const int pool[3], void* stream) {
+  if (!k || !v || !kbar || !vbar || !pool || B < 1 || heads < 1) return BASA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return BASA_ERR_UNSUPPORTED;
+  int G = 0;
+  int rc = basa_kv_pool_tokens(T, H, W, pool, &G);
+  if (rc) return rc;
+  const long long N = static_cast<long long>(T) * H * W;
+  const long long rows = static_cast<long long>(B) * N * heads;
+  const long long grows = static_cast<long long>(B) * G * heads;
+  if (rows >= (1LL << 31)) return BASA_ERR_UNSUPPORTED;
+  const void* ptrs[4] = {k, v, kbar, vbar};
+  for (const void* ptr : ptrs)
+    if (reinterpret_cast<uintptr_t>(ptr) & 15) return BASA_ERR_ALIGNMENT;
+  const size_t in_bytes = static_cast<size_t>(rows) * d * 2, out_bytes = static_cast<size_t>(grows) * d * 2;
+  if (overlaps2(kbar, out_bytes, k, in_bytes) || overlaps2(kbar, out_bytes, v, in_bytes) ||
+      overlaps2(vbar, out_bytes, k, in_bytes) || overlaps2(vbar, out_bytes, v, in_bytes) ||
+      overlaps2(kbar, out_bytes, vbar, out_bytes))
+    return BASA_ERR_ALIAS;
+  int dev = 0;
+  rc = prepare_device(&dev);
+  if (rc) return rc;
+  PoolParams pp;
+  pp.B = B;
+  pp.heads = heads;
+  pp.d = d;
+  pp.T = T;
+  pp.H = H;
+  pp.W = W;
+  const int n[3] = {T, H, W};
+  for (int a = 0; a < 3; ++a) {
+    pp.pool[a] = pool[a];
+    pp.G[a] = (n[a] + pool[a] - 1) / pool[a];
+  }
+  pp.total = grows * (d / 8);
+  const long long want = (pp.total + 255) / 256;
+  const long long cap = 8LL * g_sm_count[dev];
+  const unsigned blocks = static_cast<unsigned>(want < cap ? want : cap);
+  for (int t = 0; t < 2; ++t) {
+    pp.x = static_cast<const __nv_bfloat16*>(t == 0 ? k : v);
+    pp.xbar = static_cast<__nv_bfloat16*>(t == 0 ? kbar : vbar);
+    kv_pool_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(pp);
+  }
+  return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;
 }
 
 extern "C" int basa_shift_schedule(int L, const int win[3], const int step_offset[3], int* shifts) {

@@ -146,3 +146,32 @@ def test_shift_schedule_argument_errors(lib):
     assert lib.basa_shift_schedule(4, I3(1, 8, 8), z, None) == sw.BASA_ERR_INVALID_ARG
     with pytest.raises(sw.SwattnError):
         sw.shift_schedule(0, (1, 8, 8))
+
+
+def test_kv_pool_tokens_equal_oracle(lib):
+    for grid in ((1, 64, 64), (21, 60, 104), (3, 10, 13), (2, 5, 7)):
+        for pool in ((1, 4, 4), (1, 2, 3), (2, 4, 4), (3, 10, 13), (1, 1, 1)):
+            assert sw.kv_pool_tokens(grid, pool) == oracle.n_pooled(*grid, pool)
+
+
+def test_memory_entry_points_reject_bad_arguments_on_the_host(lib):
+    vp = ctypes.c_void_p
+    a = vp(1 << 20)          # never dereferenced: every call below fails validation first
+    win, shift, pool = I3(1, 4, 4), I3(0, 0, 0), I3(1, 2, 2)
+    E = sw.BASA_ERR_INVALID_ARG
+    # forward with memory
+    assert lib.basa_swattn_fwd_mem(a, a, a, None, None, 8, vp(1 << 24), 1, 1, 1, 8, 8, 128, win, shift, 0.1, None) == E
+    assert lib.basa_swattn_fwd_mem(a, a, a, a, a, -1, vp(1 << 24), 1, 1, 1, 8, 8, 128, win, shift, 0.1, None) == E
+    assert lib.basa_swattn_fwd_mem(a, a, a, vp((1 << 20) + 8), a, 4, vp(1 << 24), 1, 1, 1, 8, 8, 128, win, shift,
+                                   0.1, None) == sw.BASA_ERR_ALIGNMENT
+    assert lib.basa_swattn_fwd_mem(a, a, a, vp(1 << 24), a, 4, vp(1 << 24), 1, 1, 1, 8, 8, 128, win, shift,
+                                   0.1, None) == sw.BASA_ERR_ALIAS
+    assert lib.basa_swattn_fwd_mem(a, a, a, a, a, 4, vp(1 << 24), 1, 1, 1, 8, 8, 96, win, shift, 0.1,
+                                   None) == sw.BASA_ERR_UNSUPPORTED
+    # pooling
+    assert lib.basa_kv_pool(a, a, None, a, 1, 1, 1, 8, 8, 128, pool, None) == E
+    assert lib.basa_kv_pool(a, a, vp(1 << 24), vp(1 << 25), 1, 1, 1, 8, 8, 128, I3(1, 0, 2), None) == E
+    assert lib.basa_kv_pool(a, a, vp(1 << 24), vp(1 << 25), 1, 1, 1, 8, 8, 96, pool, None) == sw.BASA_ERR_UNSUPPORTED
+    assert lib.basa_kv_pool(a, a, vp((1 << 24) + 4), vp(1 << 25), 1, 1, 1, 8, 8, 128, pool,
+                            None) == sw.BASA_ERR_ALIGNMENT
+    assert lib.basa_kv_pool(a, a, a, vp(1 << 25), 1, 1, 1, 8, 8, 128, pool, None) == sw.BASA_ERR_ALIAS

@@ -208,3 +208,79 @@ def test_shift_schedule_layers(d, grid, win, L):
         out = _run_gpu(q, k, v, grid, win, shift, scale).float().cpu().numpy()
         ref = oracle.swattn_fwd(q, k, v, 1, 2, T, H, W, d, win, shift, scale)
         _check(out, ref, f"schedule layer shift={shift}")
+
+
+# ---------------------------------------------------------------- pooled global memory (§3.2)
+
+@pytest.mark.parametrize("d,grid,pool", [
+    (128, (1, 24, 24), (1, 4, 4)),
+    (64, (3, 10, 13), (2, 4, 4)),       # temporal pooling, truncated patches along t, h, w
+    (128, (2, 9, 20), (1, 3, 7)),
+])
+def test_kv_pool_matches_oracle(d, grid, pool):
+    T, H, W = grid
+    q, k, v = make_custom(2, 3, d, T, H, W, seed=sum(pool))
+    kbar, vbar = sw.kv_pool(k.cuda(), v.cuda(), grid, pool)
+    torch.cuda.synchronize()
+    for got, x in ((kbar, k), (vbar, v)):
+        ref = oracle.kv_pool(x, 2, 3, T, H, W, d, pool)
+        g = got.float().cpu().numpy().astype(np.float64)
+        # fp32 sums rounded to bf16 once: within half a bf16 ulp of the exact mean
+        assert np.all(np.abs(g - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-6)
+
+
+def _extra(B, E, heads, d, seed):
+    kx, vx, _ = make_custom(B, heads, d, 1, 1, E, seed=seed)
+    return kx, vx
+
+
+@pytest.mark.parametrize("B,heads,d,grid,win,shift,E", [
+    (1, 2, 128, (2, 9, 20), (2, 9, 7), (1, 4, 3), 37),       # pair kernel, one partial extra tile
+    (1, 2, 128, (1, 24, 24), (1, 8, 8), (0, 4, 4), 300),     # three extra tiles, the last partial
+    (2, 1, 128, (1, 16, 16), (1, 16, 16), (0, 0, 0), 128),   # full attention plus one exact extra tile
+    (1, 2, 64, (3, 10, 13), (2, 4, 5), (1, 3, 2), 77),       # one-CTA kernel (d = 64)
+])
+def test_fwd_with_extra_segment_matches_oracle(B, heads, d, grid, win, shift, E):
+    T, H, W = grid
+    q, k, v = make_custom(B, heads, d, T, H, W, seed=E)
+    kx, vx = _extra(B, E, heads, d, seed=1000 + E)
+    scale = 1.0 / math.sqrt(d)
+    dev = torch.device("cuda:0")
+    out = sw.swattn_fwd_mem(q.to(dev), k.to(dev), v.to(dev), kx.to(dev), vx.to(dev), grid, win, shift, scale)
+    assert sw.last_device_error() == sw.BASA_OK
+    ref = oracle.swattn_fwd_mem(q, k, v, kx, vx, E, B, heads, T, H, W, d, win, shift, scale)
+    _check(out.float().cpu().numpy(), ref, f"extra E={E} grid={grid} win={win} d={d}")
+
+
+def test_fwd_with_empty_extra_segment_is_bitwise_the_plain_forward():
+    grid, win, shift, d = (1, 24, 24), (1, 8, 8), (0, 4, 4), 128
+    q, k, v = make_custom(1, 2, d, *grid, seed=5)
+    dev = torch.device("cuda:0")
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    empty = torch.empty((1, 0, 2, d), dtype=torch.bfloat16, device=dev)
+    a = sw.swattn_fwd_mem(qd, kd, vd, empty, empty, grid, win, shift)
+    b = sw.swattn_fwd(qd, kd, vd, grid, win, shift)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("d,grid,win,shift,pool", [
+    (128, (1, 32, 32), (1, 8, 8), (0, 4, 4), (1, 4, 4)),         # the pages' FLUX setting (p = 4), small grid
+    (128, (3, 12, 20), (3, 6, 10), (0, 3, 5), (1, 4, 4)),        # video: full temporal extent, spatial pooling
+])
+def test_pooled_memory_pipeline(d, grid, win, shift, pool):
+    # GPU: kv_pool then the forward with the pooled tokens; oracle: its own pooling,
+    # rounded to bf16 the way every K/V operand is, then its forward
+    T, H, W = grid
+    B, heads = 1, 2
+    q, k, v = make_custom(B, heads, d, T, H, W, seed=7)
+    dev = torch.device("cuda:0")
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    kbar, vbar = sw.kv_pool(kd, vd, grid, pool)
+    out = sw.swattn_fwd_mem(qd, kd, vd, kbar, vbar, grid, win, shift)
+    assert sw.last_device_error() == sw.BASA_OK
+    G = oracle.n_pooled(T, H, W, pool)
+    kb = oracle.round_to_bf16_bits(oracle.kv_pool(k, B, heads, T, H, W, d, pool))
+    vb = oracle.round_to_bf16_bits(oracle.kv_pool(v, B, heads, T, H, W, d, pool))
+    ref = oracle.swattn_fwd_mem(q, k, v, kb, vb, G, B, heads, T, H, W, d, win, shift, 1.0 / math.sqrt(d))
+    _check(out.float().cpu().numpy(), ref, f"pooled memory grid={grid} pool={pool}")
