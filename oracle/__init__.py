@@ -7,7 +7,8 @@ code with it.
 
 The arithmetic lives in ``ref_swattn.c`` (plain C, fp64, one materialised array
 per stage), including the pooled global memory of §3.2 ("K/V-Pooled Global
-Memory").  This module only builds that file with gcc and marshals arguments
+Memory") and the true-window routing of §3.3 ("Content-Adaptive True-Window
+Routing").  This module only builds that file with gcc and marshals arguments
 through ctypes.  Method: "Backend-Agnostic Sparse Attention for Fast
 High-Resolution Visual Generation" (BASA), §3.1 "Shifted Window Sparse
 Attention" and Appendix A.1 "Regular execution with standard attention
@@ -65,6 +66,13 @@ def _load():
             lib.oref_swattn_fwd_mem.restype = ctypes.c_int
             lib.oref_kv_pool.argtypes = [ctypes.c_void_p, ctypes.c_void_p] + [ctypes.c_int] * 6 + [_I3]
             lib.oref_kv_pool.restype = ctypes.c_int
+            lib.oref_route.argtypes = ([ctypes.c_void_p, ctypes.c_void_p] + [ctypes.c_int] * 6 +
+                                       [_I3, _I3, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p])
+            lib.oref_route.restype = ctypes.c_int
+            lib.oref_swattn_fwd_route.argtypes = (
+                [ctypes.c_void_p] * 6 + [ctypes.c_int, ctypes.c_void_p] + [ctypes.c_int] * 6 +
+                [_I3, _I3, ctypes.c_double])
+            lib.oref_swattn_fwd_route.restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -213,6 +221,55 @@ def swattn_fwd_mem(q, k, v, kx, vx, E, B, heads, T, H, W, d, win, shift, scale, 
                                  int(heads), int(nthreads))
     if rc != 0:
         raise ValueError(f"oref_swattn_fwd_mem failed ({rc})")
+    return out
+
+
+def route(q, k, B, heads, T, H, W, d, win, shift, radius=1, with_scores=False):
+    """int32 [B, heads, n_windows]: the routed window of every window of the
+    (shifted) partition, -1 where a window has no candidate (§3.3: top-1 of
+    s_ij = q_i k_j^T / sqrt(d) over the other windows of the same temporal
+    index within spatial window distance `radius`).  With with_scores, also
+    the fp64 scores [B, heads, n_windows, n_windows] (-inf off the candidates)."""
+    lib = _load()
+    qb, kb = _bits(q), _bits(k)
+    nw = n_windows(T, H, W, win)
+    routed = np.full((int(B), int(heads), nw), -2, dtype=np.int32)
+    scores = np.full((int(B), int(heads), nw, nw), np.nan) if with_scores else None
+    w3, s3 = _geom_args(win, shift)
+    rc = lib.oref_route(qb.ctypes.data, kb.ctypes.data, int(B), int(heads), int(T), int(H), int(W),
+                        int(d), w3, s3, int(radius), routed.ctypes.data,
+                        scores.ctypes.data if with_scores else None)
+    if rc != 0:
+        raise ValueError(f"oref_route failed ({rc})")
+    return (routed, scores) if with_scores else routed
+
+
+def swattn_fwd_route(q, k, v, routed, kx, vx, E, B, heads, T, H, W, d, win, shift, scale):
+    """fp64 [B, T*H*W, heads, d]: every window attends to its own tokens, the
+    tokens of its routed window (routed int32 [B, heads, n_windows], -1 = none)
+    and the E extra tokens kx, vx (bf16 [B, E, heads, d]; E may be 0):
+    the key/value source S_i = W_i u R_i u G of §3.3."""
+    lib = _load()
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    nw = n_windows(T, H, W, win)
+    rt = np.ascontiguousarray(np.asarray(routed, dtype=np.int32))
+    if rt.size != int(B) * int(heads) * nw:
+        raise ValueError("routed must hold B*heads*n_windows entries")
+    if int(E) > 0:
+        kxb, vxb = _bits(kx), _bits(vx)
+        if kxb.size != int(B) * int(E) * int(heads) * int(d) or vxb.size != kxb.size:
+            raise ValueError("kx/vx must hold B*E*heads*d elements")
+        kxp, vxp = kxb.ctypes.data, vxb.ctypes.data
+    else:
+        kxp = vxp = None
+    N = int(T) * int(H) * int(W)
+    out = np.full((int(B), N, int(heads), int(d)), np.nan, dtype=np.float64)
+    w3, s3 = _geom_args(win, shift)
+    rc = lib.oref_swattn_fwd_route(qb.ctypes.data, kb.ctypes.data, vb.ctypes.data, rt.ctypes.data,
+                                   kxp, vxp, int(E), out.ctypes.data, int(B), int(heads), int(T),
+                                   int(H), int(W), int(d), w3, s3, float(scale))
+    if rc != 0:
+        raise ValueError(f"oref_swattn_fwd_route failed ({rc})")
     return out
 
 

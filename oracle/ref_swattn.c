@@ -46,6 +46,11 @@
  *   [K_W; K_bar] and [V_W; V_bar] (oref_kv_pool builds the means,
  *   oref_swattn_fwd_mem attends over a window plus any extra segment).
  *
+ *   §3.3 "Content-Adaptive True-Window Routing": window descriptors are the
+ *   means of Q and K over each window, s_ij = q_i k_j^T / sqrt(d) over a
+ *   candidate neighbourhood, the top-1 window is routed (oref_route), and each
+ *   window attends to S_i = W_i u R_i u G (oref_swattn_fwd_route).
+ *
  * Data layout: Q, K, V are bf16 [B, T*H*W, heads, d] (raster token order t,h,w),
  * passed as uint16 bit patterns; the output is fp64 [B, T*H*W, heads, d].
  */
@@ -624,4 +629,217 @@ int oref_kv_pool(const uint16_t *x, double *xbar, int B, int heads, int T, int H
                 }
         }
     return OREF_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* true-window routing (§3.3 "Content-Adaptive True-Window Routing")   */
+/* ------------------------------------------------------------------ */
+
+/*
+ * routed[b, head, i] for every window i of the layer's (shifted) partition:
+ * q_i = mean of Q over window i's tokens, k_j = mean of K over window j's
+ * tokens, s_ij = q_i . k_j / sqrt(d), separately for every head and batch
+ * item.  Routing is spatial: the candidates of i are the other windows with
+ * the same temporal window index m_t whose spatial window coordinates
+ * (m_h, m_w) are within Chebyshev distance `radius` of i's (no wrap-around:
+ * the window grid has edges).  routed is the candidate with the largest s_ij
+ * (the lowest window index on a tie), or -1 when there is none (K = 1).
+ * Computed stage by stage: roll, partition, window means, scores.
+ * q, k: bf16 [B, N, heads, d]; routed: int32 [B, heads, nW]; scores (may be
+ * NULL): fp64 [B, heads, nW, nW], s_ij for the candidates, -inf elsewhere.
+ */
+int oref_route(const uint16_t *q, const uint16_t *k, int B, int heads, int T, int H, int W, int d,
+               const int win[3], const int shift[3], int radius, int32_t *routed, double *scores)
+{
+    geom_t g;
+    long N, tok, c, wsz;
+    int b, hd, rc, m, j;
+    double *xq = NULL, *xk = NULL, *rq = NULL, *rk = NULL, *wq = NULL, *wk = NULL;
+    double *mq = NULL, *mk = NULL;
+    int *count = NULL;
+    rc = geom_init(&g, T, H, W, win, shift);
+    if (rc) return rc;
+    if (!q || !k || !routed || B < 1 || heads < 1 || d < 1 || radius < 0) return OREF_ERR_ARG;
+    N = g.N;
+    wsz = g.n_windows * g.nw_max * d;
+    xq = (double *)malloc(sizeof(double) * (size_t)(N * d));
+    xk = (double *)malloc(sizeof(double) * (size_t)(N * d));
+    rq = (double *)malloc(sizeof(double) * (size_t)(N * d));
+    rk = (double *)malloc(sizeof(double) * (size_t)(N * d));
+    wq = (double *)calloc((size_t)wsz, sizeof(double));
+    wk = (double *)calloc((size_t)wsz, sizeof(double));
+    mq = (double *)malloc(sizeof(double) * (size_t)(g.n_windows * d));
+    mk = (double *)malloc(sizeof(double) * (size_t)(g.n_windows * d));
+    count = (int *)malloc(sizeof(int) * (size_t)g.n_windows);
+    rc = OREF_OK;
+    if (!xq || !xk || !rq || !rk || !wq || !wk || !mq || !mk || !count) { rc = OREF_ERR_NOMEM; goto done; }
+    for (b = 0; b < B; ++b) {
+        for (hd = 0; hd < heads; ++hd) {
+            for (tok = 0; tok < N; ++tok) {
+                long src = (((long)b * N + tok) * heads + hd) * d;
+                for (c = 0; c < d; ++c) {
+                    xq[tok * d + c] = bf16_to_f64(q[src + c]);
+                    xk[tok * d + c] = bf16_to_f64(k[src + c]);
+                }
+            }
+            roll_grid(xq, rq, &g, d, -1);
+            roll_grid(xk, rk, &g, d, -1);
+            partition_grid(rq, wq, count, &g, d, 1);
+            partition_grid(rk, wk, NULL, &g, d, 1);
+            /* window means */
+            for (m = 0; m < g.n_windows; ++m) {
+                int s;
+                for (c = 0; c < d; ++c) {
+                    double aq = 0.0, ak = 0.0;
+                    for (s = 0; s < count[m]; ++s) {
+                        aq += wq[((long)m * g.nw_max + s) * d + c];
+                        ak += wk[((long)m * g.nw_max + s) * d + c];
+                    }
+                    mq[(long)m * d + c] = aq / count[m];
+                    mk[(long)m * d + c] = ak / count[m];
+                }
+            }
+            /* scores over the radius neighbourhood, top-1 */
+            for (m = 0; m < g.n_windows; ++m) {
+                const int mw = m % g.nwin[2], mh = (m / g.nwin[2]) % g.nwin[1], mt = m / (g.nwin[2] * g.nwin[1]);
+                int best = -1;
+                double best_s = -INFINITY;
+                double *srow = scores ? scores + (((long)b * heads + hd) * g.n_windows + m) * g.n_windows : NULL;
+                for (j = 0; j < g.n_windows; ++j) {
+                    const int jw = j % g.nwin[2], jh = (j / g.nwin[2]) % g.nwin[1], jt = j / (g.nwin[2] * g.nwin[1]);
+                    double s = 0.0;
+                    if (srow) srow[j] = -INFINITY;
+                    if (j == m || jt != mt || abs(jh - mh) > radius || abs(jw - mw) > radius)
+                        continue;
+                    for (c = 0; c < d; ++c) s += mq[(long)m * d + c] * mk[(long)j * d + c];
+                    s /= sqrt((double)d);
+                    if (srow) srow[j] = s;
+                    if (s > best_s) { best_s = s; best = j; }
+                }
+                routed[((long)b * heads + hd) * g.n_windows + m] = best;
+            }
+        }
+    }
+done:
+    free(xq); free(xk); free(rq); free(rk); free(wq); free(wk); free(mq); free(mk); free(count);
+    return rc;
+}
+
+/*
+ * The forward where window i's queries attend to the tokens of window i, of
+ * window routed[b, head, i] (when >= 0; the routed window's own tokens, in its
+ * own raster order) and of the extra segment kx, vx ([B, E, heads, d], E >= 0):
+ * the key/value source S_i = W_i u R_i u G of §3.3.  Stage by stage as the
+ * plain forward; out is fp64 [B, N, heads, d].
+ */
+int oref_swattn_fwd_route(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                          const int32_t *routed, const uint16_t *kx, const uint16_t *vx, int E,
+                          double *out, int B, int heads, int T, int H, int W, int d,
+                          const int win[3], const int shift[3], double scale)
+{
+    geom_t g;
+    long N, tok, c, wsz;
+    int b, hd, rc, m;
+    double *xq = NULL, *xk = NULL, *xv = NULL, *rq = NULL, *rk = NULL, *rv = NULL;
+    double *wq = NULL, *wk = NULL, *wv = NULL, *wo = NULL, *ro = NULL, *y = NULL;
+    double *kk = NULL, *vv = NULL, *work = NULL;
+    int *count = NULL;
+    rc = geom_init(&g, T, H, W, win, shift);
+    if (rc) return rc;
+    if (!q || !k || !v || !routed || !out || B < 1 || heads < 1 || d < 1 || E < 0 ||
+        (E > 0 && (!kx || !vx)))
+        return OREF_ERR_ARG;
+    N = g.N;
+    wsz = g.n_windows * g.nw_max * d;
+    xq = (double *)malloc(sizeof(double) * (size_t)(N * d));
+    xk = (double *)malloc(sizeof(double) * (size_t)(N * d));
+    xv = (double *)malloc(sizeof(double) * (size_t)(N * d));
+    rq = (double *)malloc(sizeof(double) * (size_t)(N * d));
+    rk = (double *)malloc(sizeof(double) * (size_t)(N * d));
+    rv = (double *)malloc(sizeof(double) * (size_t)(N * d));
+    ro = (double *)malloc(sizeof(double) * (size_t)(N * d));
+    y = (double *)malloc(sizeof(double) * (size_t)(N * d));
+    wq = (double *)calloc((size_t)wsz, sizeof(double));
+    wk = (double *)calloc((size_t)wsz, sizeof(double));
+    wv = (double *)calloc((size_t)wsz, sizeof(double));
+    wo = (double *)calloc((size_t)wsz, sizeof(double));
+    kk = (double *)malloc(sizeof(double) * (size_t)((2 * g.nw_max + E) * d));
+    vv = (double *)malloc(sizeof(double) * (size_t)((2 * g.nw_max + E) * d));
+    work = (double *)malloc(sizeof(double) * (size_t)(2 * g.nw_max + E));
+    count = (int *)malloc(sizeof(int) * (size_t)g.n_windows);
+    rc = OREF_OK;
+    if (!xq || !xk || !xv || !rq || !rk || !rv || !ro || !y || !wq || !wk || !wv || !wo || !kk || !vv ||
+        !work || !count) { rc = OREF_ERR_NOMEM; goto done; }
+    for (b = 0; b < B; ++b) {
+        for (hd = 0; hd < heads; ++hd) {
+            for (tok = 0; tok < N; ++tok) {
+                long src = (((long)b * N + tok) * heads + hd) * d;
+                for (c = 0; c < d; ++c) {
+                    xq[tok * d + c] = bf16_to_f64(q[src + c]);
+                    xk[tok * d + c] = bf16_to_f64(k[src + c]);
+                    xv[tok * d + c] = bf16_to_f64(v[src + c]);
+                }
+            }
+            roll_grid(xq, rq, &g, d, -1);
+            roll_grid(xk, rk, &g, d, -1);
+            roll_grid(xv, rv, &g, d, -1);
+            partition_grid(rq, wq, count, &g, d, 1);
+            partition_grid(rk, wk, NULL, &g, d, 1);
+            partition_grid(rv, wv, NULL, &g, d, 1);
+            for (m = 0; m < g.n_windows; ++m) {
+                const int r = routed[((long)b * heads + hd) * g.n_windows + m];
+                int n = 0, s, e;
+                /* key/value source: window m, then window r, then the extra segment */
+                for (s = 0; s < count[m]; ++s, ++n) {
+                    memcpy(kk + (long)n * d, wk + ((long)m * g.nw_max + s) * d, sizeof(double) * (size_t)d);
+                    memcpy(vv + (long)n * d, wv + ((long)m * g.nw_max + s) * d, sizeof(double) * (size_t)d);
+                }
+                if (r >= 0) {
+                    if (r >= g.n_windows) { rc = OREF_ERR_ARG; goto done; }
+                    for (s = 0; s < count[r]; ++s, ++n) {
+                        memcpy(kk + (long)n * d, wk + ((long)r * g.nw_max + s) * d, sizeof(double) * (size_t)d);
+                        memcpy(vv + (long)n * d, wv + ((long)r * g.nw_max + s) * d, sizeof(double) * (size_t)d);
+                    }
+                }
+                for (e = 0; e < E; ++e, ++n) {
+                    long src = (((long)b * E + e) * heads + hd) * d;
+                    for (c = 0; c < d; ++c) {
+                        kk[(long)n * d + c] = bf16_to_f64(kx[src + c]);
+                        vv[(long)n * d + c] = bf16_to_f64(vx[src + c]);
+                    }
+                }
+                /* dense softmax attention of window m's queries over the n keys */
+                {
+                    int i, jj;
+                    for (i = 0; i < count[m]; ++i) {
+                        const double *qi = wq + ((long)m * g.nw_max + i) * d;
+                        double *oi = wo + ((long)m * g.nw_max + i) * d;
+                        double mx = -INFINITY, sum = 0.0;
+                        for (jj = 0; jj < n; ++jj) {
+                            double sc = 0.0;
+                            for (c = 0; c < d; ++c) sc += qi[c] * kk[(long)jj * d + c];
+                            work[jj] = scale * sc;
+                            if (work[jj] > mx) mx = work[jj];
+                        }
+                        for (jj = 0; jj < n; ++jj) { work[jj] = exp(work[jj] - mx); sum += work[jj]; }
+                        for (c = 0; c < d; ++c) oi[c] = 0.0;
+                        for (jj = 0; jj < n; ++jj) {
+                            const double pj = work[jj] / sum;
+                            for (c = 0; c < d; ++c) oi[c] += pj * vv[(long)jj * d + c];
+                        }
+                    }
+                }
+            }
+            partition_grid(ro, wo, NULL, &g, d, 0);
+            roll_grid(ro, y, &g, d, +1);
+            for (tok = 0; tok < N; ++tok) {
+                long dst = (((long)b * N + tok) * heads + hd) * d;
+                memcpy(out + dst, y + tok * d, sizeof(double) * (size_t)d);
+            }
+        }
+    }
+done:
+    free(xq); free(xk); free(xv); free(rq); free(rk); free(rv); free(ro); free(y);
+    free(wq); free(wk); free(wv); free(wo); free(kk); free(vv); free(work); free(count);
+    return rc;
 }

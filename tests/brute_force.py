@@ -93,3 +93,50 @@ def masked_window_attention_with_extra(q, k, v, kx, vx, T, H, W, win, shift, sca
             p /= p.sum(axis=1, keepdims=True)
             out[b, :, h, :] = p @ vv[b, :, h, :]
     return out
+
+
+def routed_windows(q, k, T, H, W, win, shift, radius):
+    """Top-1 routing restated with numpy (§3.3 "Content-Adaptive True-Window
+    Routing"): window means from the token -> window map of ``numpy.roll``,
+    candidates = other windows with the same temporal window index within spatial
+    window distance ``radius``.  Returns (routed [B, heads, nW] int, scores
+    [B, heads, nW, nW] with -inf off the candidates)."""
+    B, N, heads, d = q.shape
+    wid = window_id_of_token(T, H, W, win, shift)
+    nwin = [-(-n // w) for n, w in zip((T, H, W), win)]
+    nW = nwin[0] * nwin[1] * nwin[2]
+    onehot = (wid[None, :] == np.arange(nW)[:, None]).astype(np.float64)   # [nW, N]
+    onehot /= onehot.sum(axis=1, keepdims=True)
+    mq = np.einsum("wn,bnhd->bhwd", onehot, q)
+    mk = np.einsum("wn,bnhd->bhwd", onehot, k)
+    ct, ch, cw = np.unravel_index(np.arange(nW), nwin)
+    cand = ((ct[:, None] == ct[None, :]) & (np.abs(ch[:, None] - ch[None, :]) <= radius) &
+            (np.abs(cw[:, None] - cw[None, :]) <= radius) & ~np.eye(nW, dtype=bool))
+    scores = np.einsum("bhid,bhjd->bhij", mq, mk) / np.sqrt(d)
+    scores = np.where(cand[None, None], scores, -np.inf)
+    routed = np.where(cand.any(axis=1)[None, None], scores.argmax(axis=3), -1)
+    return routed, scores
+
+
+def masked_routed_attention(q, k, v, routed, kx, vx, T, H, W, win, shift, scale):
+    """Full attention over [K; K_x] where a query of window i may attend to the
+    keys of window i, of window routed[b, h, i] and to every extra token: the
+    source S_i = W_i u R_i u G of §3.3 as a mask over the original token order."""
+    B, N, heads, d = q.shape
+    E = kx.shape[1]
+    wid = window_id_of_token(T, H, W, win, shift)
+    kk = np.concatenate([k, kx], axis=1)
+    vv = np.concatenate([v, vx], axis=1)
+    out = np.empty_like(q)
+    for b in range(B):
+        for h in range(heads):
+            rt = np.asarray(routed)[b, h][wid]                       # routed window of each query
+            mask = (wid[:, None] == wid[None, :]) | (rt[:, None] == wid[None, :])
+            mask = np.concatenate([mask, np.ones((N, E), dtype=bool)], axis=1)
+            s = scale * (q[b, :, h, :] @ kk[b, :, h, :].T)
+            s = np.where(mask, s, -np.inf)
+            s = s - s.max(axis=1, keepdims=True)
+            p = np.exp(s)
+            p /= p.sum(axis=1, keepdims=True)
+            out[b, :, h, :] = p @ vv[b, :, h, :]
+    return out

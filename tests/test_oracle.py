@@ -367,3 +367,122 @@ def test_fwd_with_extra_segment_of_one_dominant_key():
     out = oracle.swattn_fwd_mem(qb, bits[1], bits[2], kx, vx, 1, 1, 1, T, H, W, d,
                                 (1, 2, 2), (0, 1, 1), 1.0)
     np.testing.assert_allclose(out[0, :, 0, :], np.tile(np.arange(d), (T * H * W, 1)), rtol=0, atol=1e-30)
+
+
+# ---------------------------------------------------------------- §3.3 true-window routing
+
+@pytest.mark.parametrize("grid,win,shift,radius", [
+    ((1, 12, 12), (1, 4, 4), (0, 0, 0), 1),
+    ((1, 11, 13), (1, 4, 5), (0, 3, 7), 1),      # truncated windows, shifted partition
+    ((4, 9, 10), (2, 3, 4), (1, 2, 6), 1),       # temporal windows: candidates share m_t
+    ((3, 9, 10), (3, 3, 4), (0, 1, 2), 2),       # full temporal extent, radius 2
+])
+def test_route_matches_numpy_restatement(grid, win, shift, radius):
+    from brute_force import routed_windows
+    T, H, W = grid
+    B, heads, d = 2, 3, 8
+    bits, (q, k, _) = _qkv(B, heads, d, T, H, W, seed=sum(grid) + radius)
+    got, got_s = oracle.route(bits[0], bits[1], B, heads, T, H, W, d, win, shift, radius, with_scores=True)
+    ref, ref_s = routed_windows(q, k, T, H, W, win, shift, radius)
+    np.testing.assert_allclose(got_s, ref_s, rtol=0, atol=1e-12)
+    np.testing.assert_array_equal(got, ref)
+
+
+def test_route_candidates_are_spatial_neighbours():
+    T, H, W, win = 4, 12, 15, (2, 3, 3)
+    bits, _ = _qkv(1, 2, 8, T, H, W, seed=21)
+    routed = oracle.route(bits[0], bits[1], 1, 2, T, H, W, 8, win, (1, 1, 2), 1)
+    nwin = (2, 4, 5)
+    for h in range(2):
+        for i in range(40):
+            r = int(routed[0, h, i])
+            ti, hi, wi = np.unravel_index(i, nwin)
+            tr, hr, wr = np.unravel_index(r, nwin)
+            assert r != i and tr == ti and abs(hr - hi) <= 1 and abs(wr - wi) <= 1
+
+
+def test_route_planted_pair_and_tie_rule():
+    # window 5 of a 4x4 window grid gets query mean e_0 * 2; only window 10's keys
+    # have a component along e_0 (mean 3), so 5 routes to 10 with s = 2*3/sqrt(d);
+    # every other score is exactly 0 and the lowest candidate index wins the tie
+    T, H, W, d, win = 1, 8, 8, 4, (1, 2, 2)
+    wid = np.arange(64).reshape(8, 8)
+    wid = (wid // 8 // 2) * 4 + (wid % 8) // 2
+    q = np.zeros((1, 64, 1, d)); k = np.zeros((1, 64, 1, d))
+    q[0, wid.reshape(-1) == 5, 0, 0] = 2.0
+    k[0, wid.reshape(-1) == 10, 0, 0] = 3.0
+    routed, s = oracle.route(oracle.round_to_bf16_bits(q), oracle.round_to_bf16_bits(k), 1, 1, T, H, W, d,
+                             win, (0, 0, 0), 1, with_scores=True)
+    assert routed[0, 0, 5] == 10 and s[0, 0, 5, 10] == 2.0 * 3.0 / 2.0
+    expected_ties = {0: 1, 3: 2, 12: 8, 15: 10, 10: 5, 6: 1}
+    for i, r in expected_ties.items():
+        assert routed[0, 0, i] == r, (i, routed[0, 0, i])
+
+
+def test_route_degenerate_cases():
+    bits, _ = _qkv(1, 2, 8, 2, 6, 6, seed=3)
+    # one window per temporal slice: no candidate
+    assert (oracle.route(bits[0], bits[1], 1, 2, 2, 6, 6, 8, (1, 6, 6), (0, 0, 0), 1) == -1).all()
+    # radius 0: no candidate
+    assert (oracle.route(bits[0], bits[1], 1, 2, 2, 6, 6, 8, (1, 2, 3), (0, 1, 1), 0) == -1).all()
+    # a radius covering the grid: the argmax over every other window of the slice
+    from brute_force import routed_windows
+    _, (q, k, _) = _qkv(1, 2, 8, 2, 6, 6, seed=3)
+    got = oracle.route(bits[0], bits[1], 1, 2, 2, 6, 6, 8, (1, 2, 3), (0, 1, 1), 9)
+    _, sc = routed_windows(q, k, 2, 6, 6, (1, 2, 3), (0, 1, 1), 9)
+    nW = 12
+    for i in range(nW):
+        same_t = [j for j in range(nW) if j // 6 == i // 6 and j != i]
+        assert got[0, 0, i] == same_t[int(np.argmax(sc[0, 0, i, same_t]))]
+
+
+@pytest.mark.parametrize("grid,win,shift,E", [
+    ((1, 12, 12), (1, 4, 4), (0, 2, 2), 0),
+    ((1, 11, 13), (1, 4, 5), (0, 3, 7), 6),      # truncated windows routed to each other
+    ((3, 7, 9), (3, 3, 4), (0, 1, 2), 4),        # full temporal extent
+])
+def test_fwd_route_matches_masked_attention(grid, win, shift, E):
+    from brute_force import masked_routed_attention
+    T, H, W = grid
+    B, heads, d = 2, 2, 8
+    bits, (q, k, v) = _qkv(B, heads, d, T, H, W, seed=40 + E)
+    xbits, (kx, vx, _) = _qkv(B, heads, d, 1, 1, max(E, 1), seed=140 + E)
+    kx, vx = kx[:, :E], vx[:, :E]
+    routed = oracle.route(bits[0], bits[1], B, heads, T, H, W, d, win, shift, 1)
+    routed[0, 1, 0] = -1                                     # a window with nothing routed
+    scale = 0.7 / math.sqrt(d)
+    got = oracle.swattn_fwd_route(*bits, routed, xbits[0][: B * E * heads * d] if E else None,
+                                  xbits[1][: B * E * heads * d] if E else None, E,
+                                  B, heads, T, H, W, d, win, shift, scale)
+    ref = masked_routed_attention(q, k, v, routed, kx, vx, T, H, W, win, shift, scale)
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+
+
+def test_fwd_route_with_nothing_routed_is_the_memory_forward():
+    T, H, W, d, E = 1, 6, 8, 8, 3
+    bits, _ = _qkv(1, 2, d, T, H, W, seed=4)
+    xbits, _ = _qkv(1, 2, d, 1, 1, E, seed=5)
+    none = np.full((1, 2, oracle.n_windows(T, H, W, (1, 3, 4))), -1, dtype=np.int32)
+    a = oracle.swattn_fwd_route(*bits, none, xbits[0], xbits[1], E, 1, 2, T, H, W, d, (1, 3, 4), (0, 1, 2), 0.3)
+    b = oracle.swattn_fwd_mem(*bits, xbits[0], xbits[1], E, 1, 2, T, H, W, d, (1, 3, 4), (0, 1, 2), 0.3)
+    np.testing.assert_array_equal(a, b)
+
+
+def test_fwd_route_dominant_routed_key():
+    # a key in the routed window whose logit dominates: every query of the routing
+    # window returns that key's value; windows 1 and 2 (which neither hold that key
+    # nor route to its window) do not
+    T, H, W, d, win = 1, 4, 4, 4, (1, 2, 2)
+    bits, (q, k, v) = _qkv(1, 1, d, T, H, W, seed=9, dist="uniform")
+    qb = oracle.round_to_bf16_bits(np.ones((1, 16, 1, d)))
+    kf = bf16_bits_to_f64(bits[1]).reshape(1, 16, 1, d).copy()
+    kf[0, 15] = 64.0                                         # token (3,3): window 3
+    vf = bf16_bits_to_f64(bits[2]).reshape(1, 16, 1, d).copy()
+    vf[0, 15] = np.arange(d)
+    routed = np.array([[[3, 0, 0, 1]]], dtype=np.int32)      # window 0 -> 3
+    out = oracle.swattn_fwd_route(qb, oracle.round_to_bf16_bits(kf), oracle.round_to_bf16_bits(vf), routed,
+                                  None, None, 0, 1, 1, T, H, W, d, win, (0, 0, 0), 1.0)
+    wid = window_id_of_token(T, H, W, win, (0, 0, 0))
+    np.testing.assert_allclose(out[0, wid == 0, 0, :], np.tile(np.arange(d), (4, 1)), rtol=0, atol=1e-30)
+    other = (wid == 1) | (wid == 2)
+    assert np.all(np.abs(out[0, other, 0, :] - np.arange(d)).max(axis=1) > 1e-3)
