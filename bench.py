@@ -492,6 +492,46 @@ def run_native(args):
                 "tflops_fwd": f_mem / ms_mem / 1e9,
                 "pool_gbs": 2 * (wl.B * wl.N + wl.B * G) * wl.heads * wl.d * 2 / ms_pool / 1e6}
             del kbar, vbar
+        # True-window routing (§3.3): window descriptors and top-1 routes, then
+        # the forward over S_i = W_i u R_i u G (with the pooled memory above when
+        # enabled), on the second shift of the workload.
+        if args.route:
+            import numpy as np
+            shift = wl.shifts[1]
+            nw = sw.n_windows(wl.grid, wl.win)
+            ws = torch.empty(sw.route_workspace_bytes(wl.B, wl.heads, wl.grid, wl.d, wl.win), dtype=torch.uint8,
+                             device=device)
+            routed = torch.empty((wl.B, wl.heads, nw), dtype=torch.int32, device=device)
+
+            def route_only():
+                sw.route(q, k, wl.grid, wl.win, shift, 1, out=routed, workspace=ws, stream=stream)
+            time_launches(route_only, 2, stream)
+            ms_route = statistics.median(time_launches(route_only, 10, stream))
+            pool = tuple(int(x) for x in args.memory_pool.split(",")) if args.memory_pool else None
+            G = sw.kv_pool_tokens(wl.grid, pool) if pool else 0
+            kbar, vbar = sw.kv_pool(k, v, wl.grid, pool, stream=stream) if pool else (None, None)
+
+            def fwd_route():
+                sw.swattn_fwd_route(q, k, v, routed, wl.grid, wl.win, shift, kbar, vbar, wl.scale, out=out,
+                                    stream=stream)
+            time_launches(fwd_route, 2, stream)
+            ms_fwd_rt = statistics.median(time_launches(fwd_route, 10, stream))
+            torch.cuda.synchronize()
+            # FLOPs from the routes taken: 4 d per (query, key) pair, keys = own
+            # window + routed window + G pooled tokens
+            counts = (sw.index_map_host(wl.grid, wl.win, shift) >= 0).sum(axis=1).astype(np.float64)
+            r = routed.cpu().numpy().reshape(-1, nw)
+            n_rt = np.where(r >= 0, counts[np.clip(r, 0, None)], 0.0)
+            f_rt = 4.0 * wl.d * float(np.sum(counts[None, :] * (counts[None, :] + n_rt + G)))
+            extras["route"] = {
+                "radius": 1, "top_k": 1, "shift_thw": list(shift), "windows": nw,
+                "routed_fraction": float(np.mean(r >= 0)),
+                "ms_route": ms_route,
+                "route_gbs": 2 * wl.B * wl.N * wl.heads * wl.d * 2 / ms_route / 1e6,
+                "pool_thw": list(pool) if pool else None, "pooled_tokens": G,
+                "ms_fwd": ms_fwd_rt, "flops_fwd": f_rt, "tflops_fwd": f_rt / ms_fwd_rt / 1e9,
+                "source": "own window + routed window" + (" + pooled memory" if pool else "")}
+            del ws, routed, kbar, vbar
         # CPU baseline: the oracle on a bounded sample of the same workload
         if not args.no_cpu_baseline:
             qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
@@ -546,6 +586,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end timing")
     ap.add_argument("--memory-pool", default="1,4,4",
                     help="also time the pooled global memory: pooling factors t,h,w ('' to skip)")
+    ap.add_argument("--route", action=argparse.BooleanOptionalAction, default=True,
+                    help="time true-window routing and the routed forward (the `route` key)")
     ap.add_argument("--schedule-layers", type=int, default=8,
                     help="also time an L-layer stack under the interleaved shift schedule (0: off)")
     ap.add_argument("--workload", default=HEADLINE,

@@ -34,6 +34,7 @@
 #ifndef BASA_SWATTN_H
 #define BASA_SWATTN_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -141,6 +142,57 @@ int basa_kv_pool_tokens(int T, int H, int W, const int pool[3], int* G);
  * Returns BASA_ERR_INVALID_ARG for L < 1, a window < 1 or null pointers.
  */
 int basa_shift_schedule(int L, const int win[3], const int step_offset[3], int* shifts);
+
+/*
+ * Bytes of device workspace basa_route needs: two fp32 arrays of
+ * B * heads * n_windows * d (the window descriptors).  Written to *bytes.
+ * The workspace does not depend on the shift.
+ */
+int basa_route_workspace_bytes(int B, int heads, int T, int H, int W, int d, const int win[3],
+                               size_t* bytes);
+
+/*
+ * Content-adaptive true-window routing (§3.3 "Content-Adaptive True-Window
+ * Routing"), top-1: for every window i of the shifted partition and every
+ * (batch item, head), the window descriptors q_i and k_i are the means of Q
+ * and K over the window's tokens, and routed[b, head, i] is the candidate j
+ * with the largest s_ij = q_i k_j^T / sqrt(d).  Routing is spatial (as for
+ * video in the same section): the candidates of i are the other windows with
+ * the same temporal window index whose (m_h, m_w) lie within Chebyshev
+ * distance `radius` of i's, without wrap-around.  Ties go to the lower window
+ * index; a window with no candidate (radius 0, or one spatial window) gets -1.
+ *
+ *   q, k       device bf16 [B, T*H*W, heads, d], 16-byte aligned (as basa_swattn_fwd)
+ *   workspace  device, >= basa_route_workspace_bytes(...) bytes, 16-byte
+ *              aligned; overwritten (fp32 descriptors)
+ *   routed     out: device int32 [B, heads, n_windows], 4-byte aligned
+ * Descriptors and scores are fp32 and summed in a fixed order, so the result
+ * is the same on every run; where two candidates' scores differ by less than
+ * the fp32 rounding of the sums, either may be chosen.  Two launches on
+ * `stream`.  Errors: BASA_ERR_INVALID_ARG (null pointer, radius < 0, workspace
+ * too small, bad geometry), BASA_ERR_UNSUPPORTED (d not 64/128, sizes past
+ * 2^31 rows), BASA_ERR_ALIGNMENT, BASA_ERR_ALIAS (routed or the workspace
+ * overlapping q, k or each other), BASA_ERR_CUDA.
+ */
+int basa_route(const void* q, const void* k, int B, int heads, int T, int H, int W, int d,
+               const int win[3], const int shift[3], int radius, void* workspace,
+               size_t workspace_bytes, int32_t* routed, void* stream);
+
+/*
+ * The forward over the key/value source S_i = W_i u R_i u G of §3.3: the
+ * queries of window i attend to the tokens of window i, then to the tokens of
+ * window routed[b, head, i] (its own token order; any entry outside
+ * [0, n_windows), -1 by convention, routes nothing), then to the E extra
+ * tokens kx, vx (G, e.g. the pooled memory; E = 0 allowed, kx, vx may then be
+ * null), all in one softmax.  routed: device int32 [B, heads, n_windows],
+ * 4-byte aligned, not null (from basa_route or the caller's own choice).  With
+ * every entry -1 the result is basa_swattn_fwd_mem's.  Other arguments,
+ * errors and ownership as basa_swattn_fwd_mem; out must not overlap routed.
+ */
+int basa_swattn_fwd_route(const void* q, const void* k, const void* v, const int32_t* routed,
+                          const void* kx, const void* vx, int E, void* out, int B, int heads,
+                          int T, int H, int W, int d, const int win[3], const int shift[3],
+                          float scale, void* stream);
 
 /*
  * Synchronises `stream`, then returns BASA_ERR_DEVICE if any launch since the

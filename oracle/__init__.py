@@ -73,6 +73,10 @@ def _load():
                 [ctypes.c_void_p] * 6 + [ctypes.c_int, ctypes.c_void_p] + [ctypes.c_int] * 6 +
                 [_I3, _I3, ctypes.c_double])
             lib.oref_swattn_fwd_route.restype = ctypes.c_int
+            lib.oref_swattn_rows_route.argtypes = (
+                [ctypes.c_void_p] * 6 + [ctypes.c_int] + [ctypes.c_int] * 6 +
+                [_I3, _I3, ctypes.c_double, ctypes.c_void_p, ctypes.c_long, ctypes.c_void_p])
+            lib.oref_swattn_rows_route.restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -270,6 +274,31 @@ def swattn_fwd_route(q, k, v, routed, kx, vx, E, B, heads, T, H, W, d, win, shif
                                    int(H), int(W), int(d), w3, s3, float(scale))
     if rc != 0:
         raise ValueError(f"oref_swattn_fwd_route failed ({rc})")
+    return out
+
+
+def swattn_rows_route(q, k, v, routed, kx, vx, E, B, heads, T, H, W, d, win, shift, scale, triples):
+    """fp64 rows [len(triples), d] of ``swattn_fwd_route`` for (b, token, head) triples."""
+    lib = _load()
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    rt = np.ascontiguousarray(np.asarray(routed, dtype=np.int32))
+    if rt.size != int(B) * int(heads) * n_windows(T, H, W, win):
+        raise ValueError("routed must hold B*heads*n_windows entries")
+    if int(E) > 0:
+        kxb, vxb = _bits(kx), _bits(vx)
+        if kxb.size != int(B) * int(E) * int(heads) * int(d) or vxb.size != kxb.size:
+            raise ValueError("kx/vx must hold B*E*heads*d elements")
+        kxp, vxp = kxb.ctypes.data, vxb.ctypes.data
+    else:
+        kxp = vxp = None
+    tr = np.ascontiguousarray(np.asarray(triples, dtype=np.int64).reshape(-1, 3))
+    out = np.empty((tr.shape[0], int(d)), dtype=np.float64)
+    w3, s3 = _geom_args(win, shift)
+    rc = lib.oref_swattn_rows_route(qb.ctypes.data, kb.ctypes.data, vb.ctypes.data, rt.ctypes.data, kxp, vxp,
+                                    int(E), int(B), int(heads), int(T), int(H), int(W), int(d), w3, s3,
+                                    float(scale), tr.ctypes.data, tr.shape[0], out.ctypes.data)
+    if rc != 0:
+        raise ValueError(f"oref_swattn_rows_route failed ({rc})")
     return out
 
 

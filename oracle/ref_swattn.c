@@ -843,3 +843,108 @@ done:
     free(wq); free(wk); free(wv); free(wo); free(kk); free(vv); free(work); free(count);
     return rc;
 }
+
+/*
+ * Output rows of oref_swattn_fwd_route for (b, token, head) triples only:
+ * the token's window (found by the roll by -Delta, as in oref_swattn_rows),
+ * then the tokens of its routed window routed[b, head, window] (when >= 0),
+ * then the E extra tokens, one softmax row over them, in the same operation
+ * order as oref_swattn_fwd_route.  out_rows: fp64 [nrows][d].
+ */
+int oref_swattn_rows_route(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                           const int32_t *routed, const uint16_t *kx, const uint16_t *vx, int E,
+                           int B, int heads, int T, int H, int W, int d,
+                           const int win[3], const int shift[3], double scale,
+                           const int64_t *triples, long nrows, double *out_rows)
+{
+    geom_t g;
+    long r, cap;
+    int rc = geom_init(&g, T, H, W, win, shift);
+    double *kk, *vv, *qrow, *work;
+    if (rc) return rc;
+    if (!q || !k || !v || !routed || !triples || !out_rows || B < 1 || heads < 1 || d < 1 || E < 0 ||
+        (E > 0 && (!kx || !vx)))
+        return OREF_ERR_ARG;
+    cap = 2L * g.nw_max + E;
+    kk = (double *)malloc(sizeof(double) * (size_t)cap * d);
+    vv = (double *)malloc(sizeof(double) * (size_t)cap * d);
+    qrow = (double *)malloc(sizeof(double) * (size_t)d);
+    work = (double *)malloc(sizeof(double) * (size_t)cap);
+    if (!kk || !vv || !qrow || !work) {
+        free(kk); free(vv); free(qrow); free(work);
+        return OREF_ERR_NOMEM;
+    }
+    for (r = 0; r < nrows; ++r) {
+        long b = triples[3 * r], tok = triples[3 * r + 1], hd = triples[3 * r + 2];
+        long p[3], rp[3], m[3], c, j, n, seg, wid, rt;
+        double mx = -INFINITY, sum = 0.0;
+        if (b < 0 || b >= B || tok < 0 || tok >= g.N || hd < 0 || hd >= heads) {
+            rc = OREF_ERR_ARG;
+            break;
+        }
+        p[0] = tok / ((long)g.n[1] * g.n[2]);
+        p[1] = (tok / g.n[2]) % g.n[1];
+        p[2] = tok % g.n[2];
+        for (c = 0; c < 3; ++c) {
+            rp[c] = pmod(p[c] - g.delta[c], g.n[c]);
+            m[c] = rp[c] / g.w[c];
+        }
+        wid = (m[0] * g.nwin[1] + m[1]) * g.nwin[2] + m[2];
+        rt = routed[(b * heads + hd) * g.n_windows + wid];
+        if (rt >= g.n_windows) {
+            rc = OREF_ERR_ARG;
+            break;
+        }
+        /* keys: the token's window, then the routed window, each in slot order */
+        n = 0;
+        for (seg = 0; seg < 2; ++seg) {
+            long mm[3], e[3], st, sh, sw, id = seg == 0 ? wid : rt;
+            if (id < 0) continue;
+            mm[2] = id % g.nwin[2];
+            mm[1] = (id / g.nwin[2]) % g.nwin[1];
+            mm[0] = id / ((long)g.nwin[2] * g.nwin[1]);
+            for (c = 0; c < 3; ++c) e[c] = window_extent(&g, (int)c, (int)mm[c]);
+            for (st = 0; st < e[0]; ++st)
+                for (sh = 0; sh < e[1]; ++sh)
+                    for (sw = 0; sw < e[2]; ++sw, ++n) {
+                        long ot = pmod(mm[0] * g.w[0] + st + g.delta[0], g.n[0]);
+                        long oh = pmod(mm[1] * g.w[1] + sh + g.delta[1], g.n[1]);
+                        long ow = pmod(mm[2] * g.w[2] + sw + g.delta[2], g.n[2]);
+                        long src = ((b * g.N + (ot * g.n[1] + oh) * g.n[2] + ow) * heads + hd) * d;
+                        for (c = 0; c < d; ++c) {
+                            kk[n * d + c] = bf16_to_f64(k[src + c]);
+                            vv[n * d + c] = bf16_to_f64(v[src + c]);
+                        }
+                    }
+        }
+        /* then the extra segment */
+        for (j = 0; j < E; ++j, ++n) {
+            long src = ((b * E + j) * heads + hd) * d;
+            for (c = 0; c < d; ++c) {
+                kk[n * d + c] = bf16_to_f64(kx[src + c]);
+                vv[n * d + c] = bf16_to_f64(vx[src + c]);
+            }
+        }
+        {
+            long src = ((b * g.N + tok) * heads + hd) * d;
+            for (c = 0; c < d; ++c) qrow[c] = bf16_to_f64(q[src + c]);
+        }
+        for (j = 0; j < n; ++j) {
+            double s = 0.0;
+            for (c = 0; c < d; ++c) s += qrow[c] * kk[j * d + c];
+            work[j] = scale * s;
+            if (work[j] > mx) mx = work[j];
+        }
+        for (j = 0; j < n; ++j) {
+            work[j] = exp(work[j] - mx);
+            sum += work[j];
+        }
+        for (c = 0; c < d; ++c) out_rows[r * d + c] = 0.0;
+        for (j = 0; j < n; ++j) {
+            const double pj = work[j] / sum;
+            for (c = 0; c < d; ++c) out_rows[r * d + c] += pj * vv[j * d + c];
+        }
+    }
+    free(kk); free(vv); free(qrow); free(work);
+    return rc;
+}

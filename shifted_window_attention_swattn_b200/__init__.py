@@ -17,7 +17,8 @@ import threading
 
 __all__ = [
     "swattn_fwd", "swattn_fwd_from_host", "swattn_fwd_mem", "kv_pool", "kv_pool_tokens",
-    "index_map", "index_map_host", "flops", "shift_schedule",
+    "index_map", "index_map_host", "flops", "shift_schedule", "route", "route_workspace_bytes",
+    "swattn_fwd_route", "n_windows",
     "last_device_error", "set_wait_timeout_ns", "strerror", "library_path", "SwattnError",
 ]
 
@@ -74,6 +75,12 @@ def _load():
         lib.basa_kv_pool_tokens.restype = ci
         lib.basa_shift_schedule.argtypes = [ci, _I3, _I3, vp]
         lib.basa_shift_schedule.restype = ci
+        lib.basa_route_workspace_bytes.argtypes = [ci] * 6 + [_I3, ctypes.POINTER(ctypes.c_size_t)]
+        lib.basa_route_workspace_bytes.restype = ci
+        lib.basa_route.argtypes = [vp, vp] + [ci] * 6 + [_I3, _I3, ci, vp, ctypes.c_size_t, vp, vp]
+        lib.basa_route.restype = ci
+        lib.basa_swattn_fwd_route.argtypes = [vp] * 6 + [ci, vp] + [ci] * 6 + [_I3, _I3, ctypes.c_float, vp]
+        lib.basa_swattn_fwd_route.restype = ci
         lib.basa_swattn_last_device_error.argtypes = [vp]
         lib.basa_swattn_last_device_error.restype = ci
         lib.basa_swattn_set_wait_timeout_ns.argtypes = [ctypes.c_ulonglong]
@@ -95,6 +102,16 @@ def _triple(x, what):
     if len(t) != 3:
         raise ValueError(f"{what} must be a (t, h, w) triple")
     return t
+
+
+def n_windows(grid, win) -> int:
+    """Windows in the partition of ``grid`` by ``win``: the product of ceil(n_a / w_a)."""
+    n = 1
+    for extent, w in zip(_triple(grid, "grid"), _triple(win, "win")):
+        if w < 1:
+            raise ValueError("window extents must be >= 1")
+        n *= -(-extent // w)
+    return n
 
 
 def _stream_handle(stream, device):
@@ -171,6 +188,105 @@ def swattn_fwd_mem(q, k, v, kx, vx, grid, win, shift, scale=None, out=None, stre
                                  float(scale), _stream_handle(stream, q.device))
     if rc != BASA_OK:
         raise SwattnError(rc, "basa_swattn_fwd_mem")
+    return out
+
+
+def _check_qkv(named, grid):
+    import torch
+    for name, t in named:
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or not t.is_cuda:
+            raise TypeError(f"{name} must be a bf16 CUDA tensor")
+        if not t.is_contiguous() or t.dim() != 4:
+            raise ValueError(f"{name} must be contiguous and 4-D")
+    q = named[0][1]
+    for name, t in named[1:]:
+        if t.shape != q.shape:
+            raise ValueError(f"{name} must have the shape of q")
+    T, H, W = grid
+    if q.shape[1] != T * H * W:
+        raise ValueError(f"token count {q.shape[1]} != T*H*W = {T * H * W}")
+
+
+def route_workspace_bytes(B, heads, grid, d, win) -> int:
+    """Device bytes ``route`` needs for the fp32 window descriptors."""
+    lib = _load()
+    T, H, W = _triple(grid, "grid")
+    n = ctypes.c_size_t(0)
+    rc = lib.basa_route_workspace_bytes(int(B), int(heads), T, H, W, int(d), _I3(*_triple(win, "win")),
+                                        ctypes.byref(n))
+    if rc != BASA_OK:
+        raise SwattnError(rc, "basa_route_workspace_bytes")
+    return int(n.value)
+
+
+def route(q, k, grid, win, shift, radius=1, out=None, workspace=None, stream=None):
+    """Top-1 true-window routing (§3.3): int32 CUDA tensor [B, heads, n_windows],
+    the routed window of every window of the shifted partition (-1: none).
+    q, k: bf16 CUDA tensors [B, T*H*W, heads, d].  ``workspace`` (a CUDA tensor of
+    at least ``route_workspace_bytes`` bytes) is allocated when not given."""
+    import torch
+    lib = _load()
+    T, H, W = _triple(grid, "grid")
+    w3, s3 = _triple(win, "win"), _triple(shift, "shift")
+    _check_qkv((("q", q), ("k", k)), (T, H, W))
+    B, _, heads, d = q.shape
+    nw = n_windows(grid, win)
+    need = route_workspace_bytes(B, heads, grid, d, win)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    elif not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    if out is None:
+        out = torch.empty((B, heads, nw), dtype=torch.int32, device=q.device)
+    elif out.shape != (B, heads, nw) or out.dtype != torch.int32 or not out.is_contiguous():
+        raise ValueError(f"out must be a contiguous int32 tensor of shape {(B, heads, nw)}")
+    ws_bytes = workspace.numel() * workspace.element_size()
+    rc = lib.basa_route(q.data_ptr(), k.data_ptr(), B, heads, T, H, W, d, _I3(*w3), _I3(*s3), int(radius),
+                        workspace.data_ptr(), ws_bytes, out.data_ptr(), _stream_handle(stream, q.device))
+    if rc != BASA_OK:
+        raise SwattnError(rc, "basa_route")
+    return out
+
+
+def swattn_fwd_route(q, k, v, routed, grid, win, shift, kx=None, vx=None, scale=None, out=None, stream=None):
+    """Shifted-window attention over S_i = W_i u R_i u G (§3.3): every window
+    attends to its own tokens, to those of its routed window (``routed``: int32
+    CUDA tensor [B, heads, n_windows] from ``route``; -1 = none) and, when given,
+    to the extra K/V segment kx, vx (bf16 [B, E, heads, d], e.g. the pooled memory)."""
+    import torch
+    lib = _load()
+    T, H, W = _triple(grid, "grid")
+    w3, s3 = _triple(win, "win"), _triple(shift, "shift")
+    _check_qkv((("q", q), ("k", k), ("v", v)), (T, H, W))
+    B, N, heads, d = q.shape
+    nw = n_windows(grid, win)
+    if (not isinstance(routed, torch.Tensor) or not routed.is_cuda or routed.dtype != torch.int32 or
+            not routed.is_contiguous() or routed.numel() != B * heads * nw):
+        raise ValueError(f"routed must be a contiguous int32 CUDA tensor of {B * heads * nw} entries")
+    if (kx is None) != (vx is None):
+        raise ValueError("give both kx and vx, or neither")
+    E = 0
+    if kx is not None:
+        for name, t in (("kx", kx), ("vx", vx)):
+            if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or not t.is_cuda:
+                raise TypeError(f"{name} must be a bf16 CUDA tensor")
+            if not t.is_contiguous() or t.dim() != 4:
+                raise ValueError(f"{name} must be contiguous and 4-D")
+        if kx.shape != vx.shape or kx.shape[0] != B or kx.shape[2:] != q.shape[2:]:
+            raise ValueError("kx, vx must be [B, E, heads, d] like q")
+        E = kx.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    elif out.shape != q.shape or out.dtype != torch.bfloat16 or not out.is_contiguous():
+        raise ValueError("out must be a contiguous bf16 tensor shaped like q")
+    if scale is None:
+        scale = d ** -0.5
+    rc = lib.basa_swattn_fwd_route(q.data_ptr(), k.data_ptr(), v.data_ptr(), routed.data_ptr(),
+                                   kx.data_ptr() if E else None, vx.data_ptr() if E else None, E,
+                                   out.data_ptr(), B, heads, T, H, W, d, _I3(*w3), _I3(*s3), float(scale),
+                                   _stream_handle(stream, q.device))
+    if rc != BASA_OK:
+        raise SwattnError(rc, "basa_swattn_fwd_route")
     return out
 
 

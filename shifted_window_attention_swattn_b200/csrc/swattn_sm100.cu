@@ -143,6 +143,7 @@ struct __align__(64) FwdParams {
   CUtensorMap tq, tk, tv;       // 2D [rows = B*N*heads, cols = d], box {64, 1}, 128B swizzle
   CUtensorMap tkx, tvx;         // extra K/V segment, 2D [rows = B*n_extra*heads, cols = d] (kMem)
   int n_extra;                  // extra keys appended to every window (kMem)
+  const int* routed;            // [B, heads, n_windows] routed window of each window, or none (kRoute)
   __nv_bfloat16* out;
   Geometry g;
   int B, heads, d;
@@ -191,21 +192,39 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Sm
 }
 
 // One unit of work: up to 256 queries (two 128-row tiles) of one window of
-// one (batch item, head), attending to every key of that window.
+// one (batch item, head), attending to every key of that window, then (kRoute)
+// to every key of its routed window, then (kMem) to the extra segment.
 struct Unit {
   int b, h;
   int m[3], e[3];
   int n_valid;    // tokens in the window
   int q0;         // first query slot of tile 0
-  int nkv;        // key tiles: the window's, then (kMem) those of the extra segment
+  int nkv;        // key tiles: the window's, the routed window's (kRoute), the extra segment's (kMem)
   int nkv_win;    // key tiles of the window
+  int nkv_rt;     // key tiles of the routed window (kRoute), else 0
+  int rm[3], re[3];  // coordinates and extents of the routed window (kRoute)
+  int n_route;    // tokens of the routed window (kRoute), else 0
   int n_extra;    // keys of the extra segment (kMem), else 0
   bool has_q1;    // tile 1 holds at least one query
 };
 
+// The routed window of window win_id for the unit's (b, head): an entry
+// outside [0, n_windows) (-1 by convention) routes nothing.
+__device__ __forceinline__ void route_of(const Geometry& g, const int* routed, int heads, int win_id,
+                                         Unit& U) {
+  const int r = __ldg(routed + (static_cast<long long>(U.b) * heads + U.h) * g.n_windows + win_id);
+  U.n_route = 0;
+  U.nkv_rt = 0;
+  if (r >= 0 && r < g.n_windows) {
+    window_of(g, r, U.rm, U.re);
+    U.n_route = U.re[0] * U.re[1] * U.re[2];
+    U.nkv_rt = (U.n_route + kTile - 1) / kTile;
+  }
+}
+
 // Units are numbered with the query pair fastest, then window, then
 // (batch, head), so CTAs that run at the same time share K/V in L2.
-template <bool kMem>
+template <bool kMem, bool kRoute>
 __device__ __forceinline__ bool decode_unit(const FwdParams& p, int u, Unit& U) {
   const int qp = u % p.q_pairs;
   const int r = u / p.q_pairs;
@@ -220,6 +239,11 @@ __device__ __forceinline__ bool decode_unit(const FwdParams& p, int u, Unit& U) 
   U.has_q1 = U.q0 + kTile < U.n_valid;
   U.nkv = (U.n_valid + kTile - 1) / kTile;
   U.nkv_win = U.nkv;
+  U.nkv_rt = 0;
+  if (kRoute) {
+    route_of(p.g, p.routed, p.heads, win_id, U);
+    U.nkv += U.nkv_rt;
+  }
   U.n_extra = kMem ? p.n_extra : 0;
   if (kMem) U.nkv += (p.n_extra + kTile - 1) / kTile;
   return true;
@@ -230,14 +254,31 @@ __device__ __forceinline__ int unit_row(const FwdParams& p, const Unit& U, int s
   return (U.b * p.g.N + slot_token(p.g, U.m, U.e, slot)) * p.heads + U.h;
 }
 
-// Valid keys of key tile j: the window's tiles, then (kMem) the extra segment's.
-template <bool kMem>
-__device__ __forceinline__ int kv_valid_of(const Unit& U, int j) {
-  if (kMem && j >= U.nkv_win) {
-    const int left = U.n_extra - (j - U.nkv_win) * kTile;
-    return left < kTile ? left : kTile;
+// Key tile j of a unit: segment 0 = the window's tiles, 1 = the routed
+// window's (kRoute), 2 = the extra segment's (kMem); *t0 = the first key of
+// the tile within its segment.
+template <bool kMem, bool kRoute>
+__device__ __forceinline__ int seg_of(const Unit& U, int j, int* t0) {
+  if ((kMem || kRoute) && j >= U.nkv_win) {
+    const int jr = j - U.nkv_win;
+    if (kRoute && jr < U.nkv_rt) {
+      *t0 = jr * kTile;
+      return 1;
+    }
+    *t0 = (jr - (kRoute ? U.nkv_rt : 0)) * kTile;
+    return 2;
   }
-  const int left = U.n_valid - j * kTile;
+  *t0 = j * kTile;
+  return 0;
+}
+
+// Valid keys of key tile j.
+template <bool kMem, bool kRoute>
+__device__ __forceinline__ int kv_valid_of(const Unit& U, int j) {
+  int t0;
+  const int seg = seg_of<kMem, kRoute>(U, j, &t0);
+  const int n = seg == 0 ? U.n_valid : (seg == 1 ? U.n_route : U.n_extra);
+  const int left = n - t0;
   return left < kTile ? left : kTile;
 }
 
@@ -257,34 +298,52 @@ __device__ __forceinline__ void extra_rows4(const Unit& U, int heads, int s, int
 // slot's row.  The same tokens as slot_token(), slot by slot: the first slot is
 // split into (s_t, s_h, s_w) with divisions, the next three step along the
 // raster order.
-__device__ __forceinline__ void unit_rows4(const Geometry& g, const Unit& U, int heads, int s,
-                                           int r[4]) {
-  int sw = s % U.e[2];
-  const int q = s / U.e[2];
-  int sh = q % U.e[1];
-  int st = q / U.e[1];
-  const int base_t = U.m[0] * g.w[0] + g.delta[0];
-  const int base_h = U.m[1] * g.w[1] + g.delta[1];
-  const int base_w = U.m[2] * g.w[2] + g.delta[2];
-  const int tok0 = U.b * g.N;
+__device__ __forceinline__ void win_rows4(const Geometry& g, int b, int h, const int m[3], const int e[3],
+                                          int heads, int s, int r[4]) {
+  int sw = s % e[2];
+  const int q = s / e[2];
+  int sh = q % e[1];
+  int st = q / e[1];
+  const int base_t = m[0] * g.w[0] + g.delta[0];
+  const int base_h = m[1] * g.w[1] + g.delta[1];
+  const int base_w = m[2] * g.w[2] + g.delta[2];
+  const int tok0 = b * g.N;
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
-    const bool pad = st >= U.e[0];
-    int pt = base_t + (pad ? U.e[0] - 1 : st);
-    int ph = base_h + (pad ? U.e[1] - 1 : sh);
-    int pw = base_w + (pad ? U.e[2] - 1 : sw);
+    const bool pad = st >= e[0];
+    int pt = base_t + (pad ? e[0] - 1 : st);
+    int ph = base_h + (pad ? e[1] - 1 : sh);
+    int pw = base_w + (pad ? e[2] - 1 : sw);
     if (pt >= g.n[0]) pt -= g.n[0];
     if (ph >= g.n[1]) ph -= g.n[1];
     if (pw >= g.n[2]) pw -= g.n[2];
-    r[k] = (tok0 + (pt * g.n[1] + ph) * g.n[2] + pw) * heads + U.h;
-    if (++sw == U.e[2]) {
+    r[k] = (tok0 + (pt * g.n[1] + ph) * g.n[2] + pw) * heads + h;
+    if (++sw == e[2]) {
       sw = 0;
-      if (++sh == U.e[1]) {
+      if (++sh == e[1]) {
         sh = 0;
         ++st;
       }
     }
   }
+}
+
+__device__ __forceinline__ void unit_rows4(const Geometry& g, const Unit& U, int heads, int s,
+                                           int r[4]) {
+  win_rows4(g, U.b, U.h, U.m, U.e, heads, s, r);
+}
+
+// Rows of segment seg (0 window, 1 routed window, 2 extra segment) of unit U
+// for the segment's keys s .. s+3.
+template <bool kMem, bool kRoute>
+__device__ __forceinline__ void seg_rows4(const Geometry& g, const Unit& U, int heads, int seg, int s,
+                                          int r[4]) {
+  if (kMem && seg == 2)
+    extra_rows4(U, heads, s, r);
+  else if (kRoute && seg == 1)
+    win_rows4(g, U.b, U.h, U.rm, U.re, heads, s, r);
+  else
+    unit_rows4(g, U, heads, s, r);
 }
 
 // One key step of the online softmax for the S row of this thread at TMEM
@@ -351,7 +410,7 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint3
             (accumulate || kk > 0) ? 1u : 0u);
 }
 
-template <bool kMem>
+template <bool kMem, bool kRoute>
 __global__ void __launch_bounds__(kThreads, 1) swattn_fwd_kernel(const __grid_constant__ FwdParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -409,25 +468,23 @@ __global__ void __launch_bounds__(kThreads, 1) swattn_fwd_kernel(const __grid_co
     uint32_t q_use[2] = {0, 0};
     uint32_t ld = 0;          // loads issued into the ring
     bool ok = true;
-    // extra: the tile comes from the extra K/V segment (slot0 counts its tokens).
+    // seg: the segment the tile comes from (0 window, 1 routed window, 2 extra
+    // segment); slot0 counts that segment's tokens.
     auto issue = [&](const Unit& U, int slot0, const CUtensorMap* map, uint64_t* bar, uint8_t* tile,
-                     bool extra) {
+                     int seg) {
       if (elect_one()) mbar_arrive_expect_tx(bar, half_bytes);
       __syncwarp();
       for (int n = pw + kProducers * lane; n < 32 * ncb; n += 32 * kProducers) {
         const int grp = n / ncb, c = n - grp * ncb;
         int r[4];
-        if (kMem && extra)
-          extra_rows4(U, p.heads, slot0 + 4 * grp, r);
-        else
-          unit_rows4(p.g, U, p.heads, slot0 + 4 * grp, r);
+        seg_rows4<kMem, kRoute>(p.g, U, p.heads, seg, slot0 + 4 * grp, r);
         tma_gather4(map, bar, tile + c * (kTile * 128) + grp * 512, c * 64, r[0], r[1], r[2], r[3]);
       }
       __syncwarp();
     };
     for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
       Unit U;
-      if (!decode_unit<kMem>(p, u, U)) continue;
+      if (!decode_unit<kMem, kRoute>(p, u, U)) continue;
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
         if (i == 1 && !U.has_q1) break;
@@ -436,7 +493,7 @@ __global__ void __launch_bounds__(kThreads, 1) swattn_fwd_kernel(const __grid_co
                           wait_or_abort(&ctl->q_empty[i], (q_use[i] - 1) & 1, ctl, p.timeout_ns));
           if (!ok) break;
         }
-        issue(U, U.q0 + i * kTile, &p.tq, &ctl->q_full[i], sQ + i * tile_bytes, false);
+        issue(U, U.q0 + i * kTile, &p.tq, &ctl->q_full[i], sQ + i * tile_bytes, 0);
         ++q_use[i];
       }
       for (int j = 0; ok && j < U.nkv; ++j) {
@@ -448,12 +505,10 @@ __global__ void __launch_bounds__(kThreads, 1) swattn_fwd_kernel(const __grid_co
                             wait_or_abort(&ctl->kv_empty[slot], (use - 1) & 1, ctl, p.timeout_ns));
             if (!ok) break;
           }
-          if (kMem && j >= U.nkv_win)
-            issue(U, (j - U.nkv_win) * kTile, kv == 0 ? &p.tkx : &p.tvx, &ctl->kv_full[slot],
-                  sRing + slot * tile_bytes, true);
-          else
-            issue(U, j * kTile, kv == 0 ? &p.tk : &p.tv, &ctl->kv_full[slot], sRing + slot * tile_bytes,
-                  false);
+          int t0;
+          const int seg = seg_of<kMem, kRoute>(U, j, &t0);
+          const CUtensorMap* map = (kMem && seg == 2) ? (kv == 0 ? &p.tkx : &p.tvx) : (kv == 0 ? &p.tk : &p.tv);
+          issue(U, t0, map, &ctl->kv_full[slot], sRing + slot * tile_bytes, seg);
           ++ld;
         }
       }
@@ -477,7 +532,7 @@ __global__ void __launch_bounds__(kThreads, 1) swattn_fwd_kernel(const __grid_co
       bool ok = !p.stall || wait_or_abort(&ctl->never, 0, ctl, p.timeout_ns);
       for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
         Unit U;
-        if (!decode_unit<kMem>(p, u, U)) continue;
+        if (!decode_unit<kMem, kRoute>(p, u, U)) continue;
         const int nq = U.has_q1 ? 2 : 1;
 #pragma unroll
         for (int i = 0; i < 2; ++i)
@@ -490,7 +545,7 @@ __global__ void __launch_bounds__(kThreads, 1) swattn_fwd_kernel(const __grid_co
         ++ld;
         tc_fence_after();
         {
-          const int n_s = (kv_valid_of<kMem>(U, 0) + 15) & ~15;
+          const int n_s = (kv_valid_of<kMem, kRoute>(U, 0) + 15) & ~15;
 #pragma unroll
           for (int i = 0; i < 2; ++i) {
             if (i >= nq) break;
@@ -506,7 +561,7 @@ __global__ void __launch_bounds__(kThreads, 1) swattn_fwd_kernel(const __grid_co
           if (!ok) break;
           ++ld;
           const bool more = j + 1 < U.nkv;
-          const int kvv = kv_valid_of<kMem>(U, j);
+          const int kvv = kv_valid_of<kMem, kRoute>(U, j);
 #pragma unroll
           for (int i = 0; i < 2; ++i) {
             if (i >= nq) break;
@@ -525,7 +580,7 @@ __global__ void __launch_bounds__(kThreads, 1) swattn_fwd_kernel(const __grid_co
                 ++ld;
                 tc_fence_after();
               }
-              const int n_s = (kv_valid_of<kMem>(U, j + 1) + 15) & ~15;
+              const int n_s = (kv_valid_of<kMem, kRoute>(U, j + 1) + 15) & ~15;
               issue_qk(tS[i], q_addr[i], ring_addr + slot_k * tile_bytes, d, n_s);
               umma_commit(&ctl->s_full[i]);
               if (j + 1 == U.nkv - 1) umma_commit(&ctl->q_empty[i]);
@@ -554,7 +609,7 @@ __global__ void __launch_bounds__(kThreads, 1) swattn_fwd_kernel(const __grid_co
     bool ok = true;
     for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
       Unit U;
-      if (!decode_unit<kMem>(p, u, U)) continue;
+      if (!decode_unit<kMem, kRoute>(p, u, U)) continue;
       if (wg == 1 && !U.has_q1) continue;
       float m_run = -INFINITY;   // running max of scale*log2(e)*S (possibly stale by < 8)
       float l_run = 0.0f;        // running sum of exp2(x - m_run)
@@ -565,7 +620,7 @@ __global__ void __launch_bounds__(kThreads, 1) swattn_fwd_kernel(const __grid_co
         tc_fence_after();
         float alpha;
         bool need;
-        const float rowsum = softmax_row_step(tS, kv_valid_of<kMem>(U, j), sl2, m_run, alpha, need);
+        const float rowsum = softmax_row_step(tS, kv_valid_of<kMem, kRoute>(U, j), sl2, m_run, alpha, need);
         l_run = l_run * alpha + rowsum;
         if (j > 0 && __any_sync(0xffffffffu, need)) {
           // O_i holds P V of tiles 0..j-1 (complete: S_i(j) was issued after
@@ -652,6 +707,7 @@ struct __align__(64) PairParams {
   CUtensorMap tq, tk, tv;       // 2D [rows = B*N*heads, cols = 128], box {64, 1}, 128B swizzle
   CUtensorMap tkx, tvx;         // extra K/V segment, 2D [rows = B*n_extra*heads, cols = 128] (kMem)
   int n_extra;                  // extra keys appended to every window (kMem)
+  const int* routed;            // [B, heads, n_windows] routed window of each window, or none (kRoute)
   __nv_bfloat16* out;
   Geometry g;
   int B, heads;
@@ -691,7 +747,7 @@ __device__ __forceinline__ bool pair_wait(uint64_t* bar, uint32_t parity, PairCt
 }
 
 // A pair unit: up to 512 queries; tile i of CTA c holds slots q0 + 256 i + 128 c + [0, 128).
-template <bool kMem>
+template <bool kMem, bool kRoute>
 __device__ __forceinline__ bool decode_pair_unit(const PairParams& p, int u, Unit& U) {
   const int qp = u % p.q_quads;
   const int r = u / p.q_quads;
@@ -706,6 +762,11 @@ __device__ __forceinline__ bool decode_pair_unit(const PairParams& p, int u, Uni
   U.has_q1 = U.q0 + 2 * kTile < U.n_valid;
   U.nkv = (U.n_valid + kTile - 1) / kTile;
   U.nkv_win = U.nkv;
+  U.nkv_rt = 0;
+  if (kRoute) {
+    route_of(p.g, p.routed, p.heads, win_id, U);
+    U.nkv += U.nkv_rt;
+  }
   U.n_extra = kMem ? p.n_extra : 0;
   if (kMem) U.nkv += (p.n_extra + kTile - 1) / kTile;
   return true;
@@ -718,13 +779,13 @@ __device__ __forceinline__ int pair_row(const PairParams& p, const Unit& U, int 
 
 // Keys of tile j used by the MMAs: all 128, or the valid keys rounded up to 32
 // for the last tile (each CTA then holds half of them).
-template <bool kMem>
+template <bool kMem, bool kRoute>
 __device__ __forceinline__ int pair_ns(const Unit& U, int j) {
-  const int kvv = kv_valid_of<kMem>(U, j);
+  const int kvv = kv_valid_of<kMem, kRoute>(U, j);
   return kvv == kTile ? kTile : ((kvv + 31) & ~31);
 }
 
-template <bool kMem>
+template <bool kMem, bool kRoute>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     swattn_fwd_pair_kernel(const __grid_constant__ PairParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -789,18 +850,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     // producer warp n mod P (P producer warps), which computes its own four row
     // coordinates; every lane with a gather issues it in the same instruction, so
     // a warp puts up to 32 gathers in flight per issue.
-    // extra: the rows come from the extra K/V segment (slot0 counts its tokens).
+    // seg: the segment the rows come from (0 window, 1 routed window, 2 extra
+    // segment); slot0 counts that segment's tokens.
     auto gathers = [&](const Unit& U, const CUtensorMap* map, uint32_t bar_leader, uint8_t* dst,
-                       int slot0, int count, int nblk, int blk_stride, int col0, bool extra) {
+                       int slot0, int count, int nblk, int blk_stride, int col0, int seg) {
       for (int base = 0; base < count; base += 32 * kPairProducers) {
         const int n = base + pw + kPairProducers * lane;
         if (n < count) {
           const int grp = n / nblk, blk = n - grp * nblk;
           int r[4];
-          if (kMem && extra)
-            extra_rows4(U, p.heads, slot0 + 4 * grp, r);
-          else
-            unit_rows4(p.g, U, p.heads, slot0 + 4 * grp, r);
+          seg_rows4<kMem, kRoute>(p.g, U, p.heads, seg, slot0 + 4 * grp, r);
           tma_gather4_pair(map, bar_leader, dst + grp * 512 + blk * blk_stride, col0 + 64 * blk, r[0],
                            r[1], r[2], r[3]);
         }
@@ -809,7 +868,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     };
     for (int u = cluster_id; ok && u < p.total_units; u += n_clusters) {
       Unit U;
-      if (!decode_pair_unit<kMem>(p, u, U)) continue;
+      if (!decode_pair_unit<kMem, kRoute>(p, u, U)) continue;
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
         if (i == 1 && !U.has_q1) break;
@@ -822,11 +881,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         if (leader && pw == 0 && elect_one()) mbar_arrive_expect_tx(&ctl->q_full[i], 2 * kQBytes);
         __syncwarp();
         gathers(U, &p.tq, bar, sQ + i * kQBytes, U.q0 + i * 2 * kTile + static_cast<int>(rank) * kTile, 64, 2,
-                kTile * 128, 0, false);
+                kTile * 128, 0, 0);
         ++q_use[i];
       }
       for (int j = 0; ok && j < U.nkv; ++j) {
-        const int ns = pair_ns<kMem>(U, j);
+        const int ns = pair_ns<kMem, kRoute>(U, j);
         const int half = ns >> 1;
         for (int kv = 0; kv < 2; ++kv) {
           const int slot = ld % n_slots;
@@ -841,14 +900,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             mbar_arrive_expect_tx(&ctl->kv_full[slot], static_cast<uint32_t>(ns) * 256u);
           __syncwarp();
           uint8_t* dst = sRing + slot * kPairHalfTileBytes;
-          // Tiles past the window's come from the extra segment (kMem).
-          const bool extra = kMem && j >= U.nkv_win;
-          const int t0 = extra ? (j - U.nkv_win) * kTile : j * kTile;
+          // Tiles past the window's come from the routed window (kRoute), then
+          // from the extra segment (kMem).
+          int t0;
+          const int seg = seg_of<kMem, kRoute>(U, j, &t0);
+          const bool extra = kMem && seg == 2;
           if (kv == 0)   // K: keys [rank*half, rank*half + half), both column blocks
             gathers(U, extra ? &p.tkx : &p.tk, bar, dst, t0 + static_cast<int>(rank) * half, (half >> 2) * 2, 2,
-                    64 * 128, 0, extra);
+                    64 * 128, 0, seg);
           else           // V: keys [0, ns), the column block of this CTA's half of d
-            gathers(U, extra ? &p.tvx : &p.tv, bar, dst, t0, ns >> 2, 1, 0, 64 * static_cast<int>(rank), extra);
+            gathers(U, extra ? &p.tvx : &p.tv, bar, dst, t0, ns >> 2, 1, 0, 64 * static_cast<int>(rank), seg);
           ++ld;
         }
       }
@@ -890,7 +951,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       };
       for (int u = cluster_id; ok && u < p.total_units; u += n_clusters) {
         Unit U;
-        if (!decode_pair_unit<kMem>(p, u, U)) continue;
+        if (!decode_pair_unit<kMem, kRoute>(p, u, U)) continue;
         const int nq = U.has_q1 ? 2 : 1;
 #pragma unroll
         for (int i = 0; i < 2; ++i)
@@ -904,7 +965,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
           if (i >= nq) break;
-          issue_qk(i, ring_addr + slot_k * kPairHalfTileBytes, pair_ns<kMem>(U, 0));
+          issue_qk(i, ring_addr + slot_k * kPairHalfTileBytes, pair_ns<kMem, kRoute>(U, 0));
           umma_commit_pair(&ctl->s_full[i], 3);
           if (U.nkv == 1) umma_commit_pair(&ctl->q_empty[i], 3);
         }
@@ -915,7 +976,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           if (!ok) break;
           ++ld;
           const bool more = j + 1 < U.nkv;
-          const int ns = pair_ns<kMem>(U, j);
+          const int ns = pair_ns<kMem, kRoute>(U, j);
 #pragma unroll
           for (int i = 0; i < 2; ++i) {
             if (i >= nq) break;
@@ -934,7 +995,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                 ++ld;
                 tc_fence_after();
               }
-              issue_qk(i, ring_addr + slot_k * kPairHalfTileBytes, pair_ns<kMem>(U, j + 1));
+              issue_qk(i, ring_addr + slot_k * kPairHalfTileBytes, pair_ns<kMem, kRoute>(U, j + 1));
               umma_commit_pair(&ctl->s_full[i], 3);
               if (j + 1 == U.nkv - 1) umma_commit_pair(&ctl->q_empty[i], 3);
               if (i == nq - 1) umma_commit_pair(&ctl->kv_empty[slot_k], 3);
@@ -962,7 +1023,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     bool ok = true;
     for (int u = cluster_id; ok && u < p.total_units; u += n_clusters) {
       Unit U;
-      if (!decode_pair_unit<kMem>(p, u, U)) continue;
+      if (!decode_pair_unit<kMem, kRoute>(p, u, U)) continue;
       if (wg == 1 && !U.has_q1) continue;
       float m_run = -INFINITY;
       float l_run = 0.0f;
@@ -973,7 +1034,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         tc_fence_after();
         float alpha;
         bool need;
-        const float rowsum = softmax_row_step(tS, kv_valid_of<kMem>(U, j), sl2, m_run, alpha, need);
+        const float rowsum = softmax_row_step(tS, kv_valid_of<kMem, kRoute>(U, j), sl2, m_run, alpha, need);
         l_run = l_run * alpha + rowsum;
         if (j > 0 && __any_sync(0xffffffffu, need)) {
           for (int c = 0; c < 4; ++c) {
@@ -1085,6 +1146,122 @@ __global__ void kv_pool_kernel(const PoolParams p) {
   }
 }
 
+// ------------------------------------------------------------------ true-window routing
+
+// §3.3 "Content-Adaptive True-Window Routing", descriptors: qbar, kbar[b, head,
+// window, :] = the means of Q and K over the window's tokens (fp32).  One CTA
+// of 256 threads per (b, window, head), heads fastest so that CTAs running
+// together read neighbouring 256-byte pieces of the same token rows.  Thread
+// (c, l) sums the 16-byte slice c of the window's tokens l, l + L, l + 2L, ...
+// (L = 256 / (d / 8) token lanes); the L partial sums are then added in lane
+// order, so the result does not depend on scheduling.
+struct DescParams {
+  const __nv_bfloat16 *q, *k;
+  float *qbar, *kbar;
+  Geometry g;
+  int B, heads, d;
+};
+
+constexpr int kDescThreads = 256;
+
+__global__ void __launch_bounds__(kDescThreads, 2) win_desc_kernel(const DescParams p) {
+  __shared__ float red[2][kDescThreads * 8];
+  const int chunks = p.d / 8;
+  const int lanes = kDescThreads / chunks;
+  const int c = threadIdx.x % chunks;
+  const int l = threadIdx.x / chunks;
+  const int hd = blockIdx.x % p.heads;
+  const int rest = blockIdx.x / p.heads;
+  const int win = rest % p.g.n_windows;
+  const int b = rest / p.g.n_windows;
+  int m[3], e[3];
+  window_of(p.g, win, m, e);
+  const int n = e[0] * e[1] * e[2];
+  float aq[8], ak[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) aq[i] = ak[i] = 0.0f;
+#pragma unroll 4
+  for (int s = l; s < n; s += lanes) {
+    const long long row = (static_cast<long long>(b) * p.g.N + slot_token(p.g, m, e, s)) * p.heads + hd;
+    const uint4 vq = __ldg(reinterpret_cast<const uint4*>(p.q + row * p.d) + c);
+    const uint4 vk = __ldg(reinterpret_cast<const uint4*>(p.k + row * p.d) + c);
+    const uint32_t uq[4] = {vq.x, vq.y, vq.z, vq.w}, uk[4] = {vk.x, vk.y, vk.z, vk.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      aq[2 * i] += __uint_as_float(uq[i] << 16);
+      aq[2 * i + 1] += __uint_as_float(uq[i] & 0xffff0000u);
+      ak[2 * i] += __uint_as_float(uk[i] << 16);
+      ak[2 * i + 1] += __uint_as_float(uk[i] & 0xffff0000u);
+    }
+  }
+  // red[t][l * d + channel]
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    red[0][l * p.d + c * 8 + i] = aq[i];
+    red[1][l * p.d + c * 8 + i] = ak[i];
+  }
+  __syncthreads();
+  const float inv = 1.0f / static_cast<float>(n);
+  const long long out0 = ((static_cast<long long>(b) * p.heads + hd) * p.g.n_windows + win) * p.d;
+  for (int i = threadIdx.x; i < 2 * p.d; i += kDescThreads) {
+    const int t = i / p.d, ch = i - t * p.d;
+    float acc = 0.0f;
+    for (int j = 0; j < lanes; ++j) acc += red[t][j * p.d + ch];
+    (t == 0 ? p.qbar : p.kbar)[out0 + ch] = acc * inv;
+  }
+}
+
+// §3.3 routing: for each (b, head, window i) the candidate j with the largest
+// q_i . k_j (the 1/sqrt(d) factor does not change the order), candidates being
+// the other windows of the same temporal window index whose spatial window
+// coordinates are within `radius` of i's (no wrap-around); the lowest window
+// index wins a tie, -1 when there is no candidate.  One warp per window; the
+// dot products are reduced with a fixed butterfly, so every lane sees the
+// same value.
+struct RouteParams {
+  const float *qbar, *kbar;
+  int32_t* routed;
+  Geometry g;
+  long long total;   // B * heads * n_windows
+  int d, radius;
+};
+
+__global__ void route_kernel(const RouteParams p) {
+  const long long wg = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (wg >= p.total) return;
+  const int nw = p.g.n_windows;
+  const int win = static_cast<int>(wg % nw);
+  const long long bh = wg / nw;
+  const int per = p.d / 32;   // channels per lane (d is 64 or 128)
+  float qv[4];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) qv[c] = c < per ? p.qbar[wg * p.d + lane + 32 * c] : 0.0f;
+  int m[3], e[3];
+  window_of(p.g, win, m, e);
+  const int h0 = max(0, m[1] - p.radius), h1 = min(p.g.nwin[1] - 1, m[1] + p.radius);
+  const int w0 = max(0, m[2] - p.radius), w1 = min(p.g.nwin[2] - 1, m[2] + p.radius);
+  int best = -1;
+  float best_s = -INFINITY;
+  for (int jh = h0; jh <= h1; ++jh)
+    for (int jw = w0; jw <= w1; ++jw) {
+      const int j = (m[0] * p.g.nwin[1] + jh) * p.g.nwin[2] + jw;
+      if (j == win) continue;
+      const float* kd = p.kbar + (bh * nw + j) * p.d;
+      float s = 0.0f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        if (c < per) s = fmaf(qv[c], kd[lane + 32 * c], s);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      if (s > best_s) {
+        best_s = s;
+        best = j;
+      }
+    }
+  if (lane == 0) p.routed[wg] = best;
+}
+
 __global__ void index_map_kernel(Geometry g, int32_t* tos) {
   const long long total = static_cast<long long>(g.n_windows) * g.nw_max;
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
@@ -1161,31 +1338,40 @@ static int prepare_device(int* dev_out) {
     g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
   }
   size_t smem_max = smem_bytes_for(128) > smem_bytes_for(64) ? smem_bytes_for(128) : smem_bytes_for(64);
-  if (cudaFuncSetAttribute(swattn_fwd_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem_max)) != cudaSuccess ||
-      cudaFuncSetAttribute(swattn_fwd_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem_max)) != cudaSuccess)
-    return BASA_ERR_CUDA;
+  // The four segment variants of each kernel: (kMem, kRoute).
+  const void* fwd_kernels[4] = {reinterpret_cast<const void*>(swattn_fwd_kernel<false, false>),
+                                reinterpret_cast<const void*>(swattn_fwd_kernel<true, false>),
+                                reinterpret_cast<const void*>(swattn_fwd_kernel<false, true>),
+                                reinterpret_cast<const void*>(swattn_fwd_kernel<true, true>)};
+  const void* pair_kernels[4] = {reinterpret_cast<const void*>(swattn_fwd_pair_kernel<false, false>),
+                                 reinterpret_cast<const void*>(swattn_fwd_pair_kernel<true, false>),
+                                 reinterpret_cast<const void*>(swattn_fwd_pair_kernel<false, true>),
+                                 reinterpret_cast<const void*>(swattn_fwd_pair_kernel<true, true>)};
+  for (const void* f : fwd_kernels)
+    if (cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_max)) !=
+        cudaSuccess)
+      return BASA_ERR_CUDA;
   if (cudaDeviceGetAttribute(&g_sm_count[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
       g_sm_count[dev] < 1)
     return BASA_ERR_CUDA;
-  if (cudaFuncSetAttribute(swattn_fwd_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(pair_smem_bytes())) != cudaSuccess ||
-      cudaFuncSetAttribute(swattn_fwd_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(pair_smem_bytes())) != cudaSuccess)
-    return BASA_ERR_CUDA;
+  for (const void* f : pair_kernels)
+    if (cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(pair_smem_bytes())) != cudaSuccess)
+      return BASA_ERR_CUDA;
   {
-    // How many CTA pairs fit at once (SMs that cannot be paired stay idle).
+    // How many CTA pairs fit at once (SMs that cannot be paired stay idle),
+    // the fewest over the variants so that one grid size serves them all.
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * g_sm_count[dev], 1, 1);
     cfg.blockDim = dim3(kPairThreads, 1, 1);
     cfg.dynamicSmemBytes = pair_smem_bytes();
-    int n = 0, n_mem = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, swattn_fwd_pair_kernel<false>, &cfg) != cudaSuccess || n < 1 ||
-        cudaOccupancyMaxActiveClusters(&n_mem, swattn_fwd_pair_kernel<true>, &cfg) != cudaSuccess ||
-        n_mem < 1)
-      return BASA_ERR_CUDA;
-    g_pair_clusters[dev] = n < n_mem ? n : n_mem;
+    int least = 0;
+    for (const void* f : pair_kernels) {
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, f, &cfg) != cudaSuccess || n < 1) return BASA_ERR_CUDA;
+      if (least == 0 || n < least) least = n;
+    }
+    g_pair_clusters[dev] = least;
   }
   g_dev_state[dev] = 1;
   return BASA_OK;
@@ -1218,11 +1404,21 @@ static bool overlaps2(const void* a, size_t na, const void* b, size_t nb) {
 
 using namespace swattn;
 
-// The forward with an optional extra K/V segment of E tokens per (b, head)
-// appended to every window (E = 0: the plain forward).
-static int launch_fwd(const void* q, const void* k, const void* v, const void* kx, const void* vx,
-                      int E, void* out, int B, int heads, int T, int H, int W, int d, const int win[3],
-                      const int shift[3], float scale, void* stream) {
+template <typename Kernel, typename Params>
+static int launch_variant(Kernel k00, Kernel k10, Kernel k01, Kernel k11, bool mem, bool route, unsigned grid,
+                          unsigned threads, size_t smem, void* stream, const Params& p) {
+  Kernel f = mem ? (route ? k11 : k10) : (route ? k01 : k00);
+  f<<<grid, threads, smem, static_cast<cudaStream_t>(stream)>>>(p);
+  return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;
+}
+
+// The forward with an optional routed window per window (routed != null,
+// [B, heads, n_windows] on the device) and an optional extra K/V segment of E
+// tokens per (b, head) appended to every window (routed = null, E = 0: the
+// plain forward).
+static int launch_fwd(const void* q, const void* k, const void* v, const int* routed, const void* kx,
+                      const void* vx, int E, void* out, int B, int heads, int T, int H, int W, int d,
+                      const int win[3], const int shift[3], float scale, void* stream) {
   if (!q || !k || !v || !out) return BASA_ERR_INVALID_ARG;
   if (B < 1 || heads < 1 || E < 0) return BASA_ERR_INVALID_ARG;
   if (E > 0 && (!kx || !vx)) return BASA_ERR_INVALID_ARG;
@@ -1238,12 +1434,15 @@ static int launch_fwd(const void* q, const void* k, const void* v, const void* k
   const void* ptrs[6] = {q, k, v, out, E > 0 ? kx : q, E > 0 ? vx : q};
   for (const void* ptr : ptrs)
     if (reinterpret_cast<uintptr_t>(ptr) & 15) return BASA_ERR_ALIGNMENT;
+  if (routed && (reinterpret_cast<uintptr_t>(routed) & 3)) return BASA_ERR_ALIGNMENT;
   const size_t bytes = static_cast<size_t>(rows) * d * 2;
   const size_t xbytes = static_cast<size_t>(xrows) * d * 2;
   if (overlaps(out, q, bytes) || overlaps(out, k, bytes) || overlaps(out, v, bytes))
     return BASA_ERR_ALIAS;
   if (E > 0 && (overlaps2(out, bytes, kx, xbytes) || overlaps2(out, bytes, vx, xbytes)))
     return BASA_ERR_ALIAS;
+  const size_t rbytes = static_cast<size_t>(B) * heads * g.n_windows * sizeof(int);
+  if (routed && overlaps2(out, bytes, routed, rbytes)) return BASA_ERR_ALIAS;
   const long long q_pairs = (g.nw_max + 2 * kTile - 1) / (2 * kTile);
   const long long units = static_cast<long long>(B) * heads * g.n_windows * q_pairs;
   if (units >= (1LL << 31)) return BASA_ERR_UNSUPPORTED;
@@ -1265,6 +1464,7 @@ static int launch_fwd(const void* q, const void* k, const void* v, const void* k
     if (E > 0 && (encode_rows(&pp.tkx, kx, xrows, d) || encode_rows(&pp.tvx, vx, xrows, d)))
       return BASA_ERR_CUDA;
     pp.n_extra = E;
+    pp.routed = routed;
     pp.out = static_cast<__nv_bfloat16*>(out);
     pp.g = g;
     pp.B = B;
@@ -1276,13 +1476,10 @@ static int launch_fwd(const void* q, const void* k, const void* v, const void* k
     pp.timeout_ns = g_timeout_ns;
     pp.stall = g_stall;
     const long long clusters = punits < g_pair_clusters[dev] ? punits : g_pair_clusters[dev];
-    if (E > 0)
-      swattn_fwd_pair_kernel<true><<<static_cast<unsigned>(2 * clusters), kPairThreads, pair_smem_bytes(),
-                                     static_cast<cudaStream_t>(stream)>>>(pp);
-    else
-      swattn_fwd_pair_kernel<false><<<static_cast<unsigned>(2 * clusters), kPairThreads, pair_smem_bytes(),
-                                      static_cast<cudaStream_t>(stream)>>>(pp);
-    return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;
+    return launch_variant(swattn_fwd_pair_kernel<false, false>, swattn_fwd_pair_kernel<true, false>,
+                          swattn_fwd_pair_kernel<false, true>, swattn_fwd_pair_kernel<true, true>, E > 0,
+                          routed != nullptr, static_cast<unsigned>(2 * clusters), kPairThreads,
+                          pair_smem_bytes(), stream, pp);
   }
 
   FwdParams p;
@@ -1293,6 +1490,7 @@ static int launch_fwd(const void* q, const void* k, const void* v, const void* k
   if (E > 0 && (encode_rows(&p.tkx, kx, xrows, d) || encode_rows(&p.tvx, vx, xrows, d)))
     return BASA_ERR_CUDA;
   p.n_extra = E;
+  p.routed = routed;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.g = g;
   p.B = B;
@@ -1306,26 +1504,94 @@ static int launch_fwd(const void* q, const void* k, const void* v, const void* k
   p.stall = g_stall;
   // Persistent: one CTA per SM, each walking the units with a stride of the grid.
   const long long grid = units < g_sm_count[dev] ? units : g_sm_count[dev];
-  if (E > 0)
-    swattn_fwd_kernel<true><<<static_cast<unsigned>(grid), kThreads, smem_bytes_for(d),
-                              static_cast<cudaStream_t>(stream)>>>(p);
-  else
-    swattn_fwd_kernel<false><<<static_cast<unsigned>(grid), kThreads, smem_bytes_for(d),
-                               static_cast<cudaStream_t>(stream)>>>(p);
-  return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;
+  return launch_variant(swattn_fwd_kernel<false, false>, swattn_fwd_kernel<true, false>,
+                        swattn_fwd_kernel<false, true>, swattn_fwd_kernel<true, true>, E > 0,
+                        routed != nullptr, static_cast<unsigned>(grid), kThreads, smem_bytes_for(d), stream, p);
 }
 
 extern "C" int basa_swattn_fwd(const void* q, const void* k, const void* v, void* out, int B,
                                int heads, int T, int H, int W, int d, const int win[3],
                                const int shift[3], float scale, void* stream) {
-  return launch_fwd(q, k, v, nullptr, nullptr, 0, out, B, heads, T, H, W, d, win, shift, scale, stream);
+  return launch_fwd(q, k, v, nullptr, nullptr, nullptr, 0, out, B, heads, T, H, W, d, win, shift, scale,
+                    stream);
 }
 
 extern "C" int basa_swattn_fwd_mem(const void* q, const void* k, const void* v, const void* kx,
                                    const void* vx, int E, void* out, int B, int heads, int T, int H,
                                    int W, int d, const int win[3], const int shift[3], float scale,
                                    void* stream) {
-  return launch_fwd(q, k, v, kx, vx, E, out, B, heads, T, H, W, d, win, shift, scale, stream);
+  return launch_fwd(q, k, v, nullptr, kx, vx, E, out, B, heads, T, H, W, d, win, shift, scale, stream);
+}
+
+extern "C" int basa_swattn_fwd_route(const void* q, const void* k, const void* v, const int32_t* routed,
+                                     const void* kx, const void* vx, int E, void* out, int B, int heads,
+                                     int T, int H, int W, int d, const int win[3], const int shift[3],
+                                     float scale, void* stream) {
+  if (!routed) return BASA_ERR_INVALID_ARG;
+  return launch_fwd(q, k, v, routed, kx, vx, E, out, B, heads, T, H, W, d, win, shift, scale, stream);
+}
+
+extern "C" int basa_route_workspace_bytes(int B, int heads, int T, int H, int W, int d, const int win[3],
+                                          size_t* bytes) {
+  if (!bytes || B < 1 || heads < 1) return BASA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return BASA_ERR_UNSUPPORTED;
+  const int zero[3] = {0, 0, 0};
+  Geometry g;
+  int rc = make_geometry(&g, T, H, W, win, zero);
+  if (rc) return rc;
+  *bytes = 2 * static_cast<size_t>(B) * heads * g.n_windows * d * sizeof(float);
+  return BASA_OK;
+}
+
+extern "C" int basa_route(const void* q, const void* k, int B, int heads, int T, int H, int W, int d,
+                          const int win[3], const int shift[3], int radius, void* workspace,
+                          size_t workspace_bytes, int32_t* routed, void* stream) {
+  if (!q || !k || !workspace || !routed || B < 1 || heads < 1 || radius < 0) return BASA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return BASA_ERR_UNSUPPORTED;
+  Geometry g;
+  int rc = make_geometry(&g, T, H, W, win, shift);
+  if (rc) return rc;
+  size_t need = 0;
+  rc = basa_route_workspace_bytes(B, heads, T, H, W, d, win, &need);
+  if (rc) return rc;
+  if (workspace_bytes < need) return BASA_ERR_INVALID_ARG;
+  const long long rows = static_cast<long long>(B) * g.N * heads;
+  const long long descs = static_cast<long long>(B) * heads * g.n_windows;
+  if (rows >= (1LL << 31) || descs >= (1LL << 31)) return BASA_ERR_UNSUPPORTED;
+  const void* ptrs[3] = {q, k, workspace};
+  for (const void* ptr : ptrs)
+    if (reinterpret_cast<uintptr_t>(ptr) & 15) return BASA_ERR_ALIGNMENT;
+  if (reinterpret_cast<uintptr_t>(routed) & 3) return BASA_ERR_ALIGNMENT;
+  const size_t in_bytes = static_cast<size_t>(rows) * d * 2;
+  const size_t rbytes = static_cast<size_t>(descs) * sizeof(int32_t);
+  if (overlaps2(workspace, need, q, in_bytes) || overlaps2(workspace, need, k, in_bytes) ||
+      overlaps2(routed, rbytes, q, in_bytes) || overlaps2(routed, rbytes, k, in_bytes) ||
+      overlaps2(routed, rbytes, workspace, need))
+    return BASA_ERR_ALIAS;
+  int dev = 0;
+  rc = prepare_device(&dev);
+  if (rc) return rc;
+  DescParams dp;
+  dp.q = static_cast<const __nv_bfloat16*>(q);
+  dp.k = static_cast<const __nv_bfloat16*>(k);
+  dp.qbar = static_cast<float*>(workspace);
+  dp.kbar = dp.qbar + descs * d;
+  dp.g = g;
+  dp.B = B;
+  dp.heads = heads;
+  dp.d = d;
+  win_desc_kernel<<<static_cast<unsigned>(descs), kDescThreads, 0, static_cast<cudaStream_t>(stream)>>>(dp);
+  RouteParams rp;
+  rp.qbar = dp.qbar;
+  rp.kbar = dp.kbar;
+  rp.routed = routed;
+  rp.g = g;
+  rp.total = descs;
+  rp.d = d;
+  rp.radius = radius;
+  const long long blocks = (descs * 32 + 255) / 256;
+  route_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(rp);
+  return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;
 }
 
 extern "C" int basa_swattn_index_map(int T, int H, int W, const int win[3], const int shift[3],

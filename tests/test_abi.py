@@ -175,3 +175,47 @@ def test_memory_entry_points_reject_bad_arguments_on_the_host(lib):
     assert lib.basa_kv_pool(a, a, vp((1 << 24) + 4), vp(1 << 25), 1, 1, 1, 8, 8, 128, pool,
                             None) == sw.BASA_ERR_ALIGNMENT
     assert lib.basa_kv_pool(a, a, a, vp(1 << 25), 1, 1, 1, 8, 8, 128, pool, None) == sw.BASA_ERR_ALIAS
+
+
+def test_route_workspace_bytes(lib):
+    n = ctypes.c_size_t(0)
+    assert lib.basa_route_workspace_bytes(2, 3, 4, 9, 10, 64, I3(2, 3, 4), ctypes.byref(n)) == sw.BASA_OK
+    assert n.value == 2 * 2 * 3 * oracle.n_windows(4, 9, 10, (2, 3, 4)) * 64 * 4
+    assert sw.route_workspace_bytes(1, 40, (21, 45, 80), 128, (7, 15, 16)) == 2 * 40 * 45 * 128 * 4
+    assert sw.n_windows((21, 45, 80), (7, 15, 16)) == oracle.n_windows(21, 45, 80, (7, 15, 16))
+    assert lib.basa_route_workspace_bytes(1, 1, 1, 8, 8, 96, I3(1, 4, 4), ctypes.byref(n)) == sw.BASA_ERR_UNSUPPORTED
+
+
+def test_routing_entry_points_reject_bad_arguments_on_the_host(lib):
+    vp = ctypes.c_void_p
+    a = vp(1 << 20)          # never dereferenced: every call below fails validation first
+    ws, rt = vp(1 << 24), vp(1 << 25)
+    win, shift = I3(1, 4, 4), I3(0, 0, 0)
+    E = sw.BASA_ERR_INVALID_ARG
+    need = 2 * 4 * 128 * 4   # 1 x 1 x 4 windows x d 128, two fp32 arrays
+    assert lib.basa_route(a, a, 1, 1, 1, 8, 8, 128, win, shift, 1, None, need, rt, None) == E
+    assert lib.basa_route(a, a, 1, 1, 1, 8, 8, 128, win, shift, 1, ws, need, None, None) == E
+    assert lib.basa_route(a, a, 1, 1, 1, 8, 8, 128, win, shift, -1, ws, need, rt, None) == E
+    assert lib.basa_route(a, a, 1, 1, 1, 8, 8, 128, win, shift, 1, ws, need - 1, rt, None) == E
+    assert lib.basa_route(a, a, 1, 1, 1, 8, 8, 128, I3(1, 9, 4), shift, 1, ws, need, rt, None) == E
+    assert lib.basa_route(a, a, 1, 1, 1, 8, 8, 96, win, shift, 1, ws, need, rt, None) == sw.BASA_ERR_UNSUPPORTED
+    assert lib.basa_route(a, a, 1, 1, 1, 8, 8, 128, win, shift, 1, vp((1 << 24) + 8), need, rt,
+                          None) == sw.BASA_ERR_ALIGNMENT
+    assert lib.basa_route(a, a, 1, 1, 1, 8, 8, 128, win, shift, 1, ws, need, vp((1 << 25) + 2),
+                          None) == sw.BASA_ERR_ALIGNMENT
+    assert lib.basa_route(a, a, 1, 1, 1, 8, 8, 128, win, shift, 1, ws, need, vp((1 << 20) + 64),
+                          None) == sw.BASA_ERR_ALIAS
+    assert lib.basa_route(a, a, 1, 1, 1, 8, 8, 128, win, shift, 1, ws, need, vp((1 << 24) + 64),
+                          None) == sw.BASA_ERR_ALIAS
+    # the routed forward
+    out = vp(1 << 26)
+    assert lib.basa_swattn_fwd_route(a, a, a, None, None, None, 0, out, 1, 1, 1, 8, 8, 128, win, shift, 0.1,
+                                     None) == E
+    assert lib.basa_swattn_fwd_route(a, a, a, rt, None, None, 4, out, 1, 1, 1, 8, 8, 128, win, shift, 0.1,
+                                     None) == E
+    assert lib.basa_swattn_fwd_route(a, a, a, vp((1 << 25) + 2), None, None, 0, out, 1, 1, 1, 8, 8, 128, win,
+                                     shift, 0.1, None) == sw.BASA_ERR_ALIGNMENT
+    assert lib.basa_swattn_fwd_route(a, a, a, vp((1 << 26) + 64), None, None, 0, out, 1, 1, 1, 8, 8, 128, win,
+                                     shift, 0.1, None) == sw.BASA_ERR_ALIAS
+    assert lib.basa_swattn_fwd_route(a, a, a, rt, None, None, 0, out, 1, 1, 1, 8, 8, 96, win, shift, 0.1,
+                                     None) == sw.BASA_ERR_UNSUPPORTED

@@ -486,3 +486,20 @@ def test_fwd_route_dominant_routed_key():
     np.testing.assert_allclose(out[0, wid == 0, 0, :], np.tile(np.arange(d), (4, 1)), rtol=0, atol=1e-30)
     other = (wid == 1) | (wid == 2)
     assert np.all(np.abs(out[0, other, 0, :] - np.arange(d)).max(axis=1) > 1e-3)
+
+
+@pytest.mark.parametrize("E", [0, 5])
+def test_rows_route_agree_bitwise_with_full_routed_forward(E):
+    T, H, W, d, win, shift = 2, 7, 9, 8, (1, 3, 4), (1, 2, 5)
+    B, heads = 2, 2
+    bits, (q, k, _) = _qkv(B, heads, d, T, H, W, seed=77)
+    xbits, _ = _qkv(B, heads, d, 1, 1, max(E, 1), seed=78)
+    kx = xbits[0][: B * E * heads * d] if E else None
+    vx = xbits[1][: B * E * heads * d] if E else None
+    routed = oracle.route(bits[0], bits[1], B, heads, T, H, W, d, win, shift, 1)
+    routed[1, 0, 3] = -1
+    full = oracle.swattn_fwd_route(*bits, routed, kx, vx, E, B, heads, T, H, W, d, win, shift, 0.4)
+    rng = np.random.default_rng(0)
+    triples = np.stack([rng.integers(0, B, 40), rng.integers(0, T * H * W, 40), rng.integers(0, heads, 40)], 1)
+    rows = oracle.swattn_rows_route(*bits, routed, kx, vx, E, B, heads, T, H, W, d, win, shift, 0.4, triples)
+    np.testing.assert_array_equal(rows, full[triples[:, 0], triples[:, 1], triples[:, 2]])

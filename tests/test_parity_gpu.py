@@ -284,3 +284,167 @@ def test_pooled_memory_pipeline(d, grid, win, shift, pool):
     vb = oracle.round_to_bf16_bits(oracle.kv_pool(v, B, heads, T, H, W, d, pool))
     ref = oracle.swattn_fwd_mem(q, k, v, kb, vb, G, B, heads, T, H, W, d, win, shift, 1.0 / math.sqrt(d))
     _check(out.float().cpu().numpy(), ref, f"pooled memory grid={grid} pool={pool}")
+
+
+# ---------------------------------------------------------------- true-window routing (§3.3)
+
+ROUTE_TAU = 1e-4   # score margin, relative to the row's largest |s_ij|, inside which fp32 may pick either
+
+
+def _check_routes(got, ref, scores, what=""):
+    """The GPU's routed windows against the oracle's.  Where the oracle's best
+    candidate leads the runner-up by more than the margin the two must agree;
+    elsewhere (a near tie in fp64) the GPU's choice must be a candidate within
+    the margin of the best.  Windows without candidates must get -1 on both."""
+    got = np.asarray(got).reshape(ref.shape)
+    assert np.array_equal(got == -1, ref == -1), f"{what}: candidate-less windows differ"
+    cand = np.isfinite(scores)
+    srt = np.sort(np.where(cand, scores, -np.inf), axis=-1)[..., ::-1]
+    best, second = srt[..., 0], srt[..., 1]
+    scale = np.max(np.where(cand, np.abs(scores), 0.0), axis=-1)
+    tau = ROUTE_TAU * scale + 1e-12
+    has = ref >= 0
+    with np.errstate(invalid="ignore"):          # -inf - -inf where a window has < 2 candidates
+        gap = np.where(np.isfinite(second), best - second, np.inf)
+    decisive = has & (gap > tau)
+    assert np.array_equal(got[decisive], ref[decisive]), f"{what}: routes differ on decisive windows"
+    idx = np.clip(got, 0, None)[..., None]
+    picked = np.take_along_axis(scores, idx, axis=-1)[..., 0]
+    assert np.all(~has | (np.isfinite(picked) & (picked >= best - tau))), f"{what}: invalid near-tie pick"
+    assert decisive.sum() >= 0.9 * has.sum(), f"{what}: too few decisive windows to be a test"
+    return int(decisive.sum()), int(has.sum())
+
+
+@pytest.mark.parametrize("B,heads,d,grid,win,shift,radius", [
+    (2, 3, 128, (1, 24, 24), (1, 8, 8), (0, 4, 4), 1),          # image: 3x3 windows
+    (1, 2, 64, (4, 17, 22), (2, 6, 5), (1, 3, 2), 1),           # temporal windows, truncated h and w
+    (1, 2, 128, (3, 20, 26), (3, 5, 6), (0, 2, 3), 2),          # full temporal extent, radius 2
+    (1, 2, 128, (2, 8, 8), (1, 8, 8), (1, 0, 0), 1),            # one spatial window: nothing to route
+])
+def test_route_matches_oracle(B, heads, d, grid, win, shift, radius):
+    T, H, W = grid
+    q, k, _ = make_custom(B, heads, d, T, H, W, seed=radius + d)
+    got = sw.route(q.cuda(), k.cuda(), grid, win, shift, radius).cpu().numpy()
+    ref, scores = oracle.route(q, k, B, heads, T, H, W, d, win, shift, radius, with_scores=True)
+    _check_routes(got, ref, scores, f"grid={grid} win={win} radius={radius}")
+
+
+def test_route_is_deterministic():
+    grid, win, shift = (3, 20, 26), (3, 5, 6), (0, 2, 3)
+    q, k, _ = make_custom(1, 4, 128, *grid, seed=3)
+    qd, kd = q.cuda(), k.cuda()
+    a = sw.route(qd, kd, grid, win, shift)
+    for _ in range(3):
+        assert torch.equal(a, sw.route(qd, kd, grid, win, shift))
+
+
+@pytest.mark.parametrize("wl", WORKLOADS[1:], ids=lambda w: w.name)
+def test_route_full_size_workloads(wl):
+    q, k, _ = make_qkv(wl)
+    shift = wl.shifts[-1]
+    got = sw.route(q.cuda(), k.cuda(), wl.grid, wl.win, shift).cpu().numpy()
+    ref, scores = oracle.route(q, k, wl.B, wl.heads, *wl.grid, wl.d, wl.win, shift, 1, with_scores=True)
+    _check_routes(got, ref, scores, wl.name)
+
+
+def _oracle_routes(q, k, B, heads, grid, d, win, shift):
+    routed = oracle.route(q, k, B, heads, *grid, d, win, shift, 1)
+    routed[0, 0, 0] = -1            # one window with nothing routed
+    return routed
+
+
+@pytest.mark.parametrize("B,heads,d,grid,win,shift,E", [
+    (1, 2, 128, (1, 24, 24), (1, 8, 8), (0, 4, 4), 0),          # pair kernel, one partial routed tile
+    (1, 2, 128, (2, 9, 20), (2, 9, 7), (1, 4, 3), 37),          # truncated windows routed to full ones
+    (1, 2, 128, (1, 40, 40), (1, 20, 20), (0, 10, 10), 0),      # four tiles per window, ragged
+    (1, 1, 128, (1, 48, 48), (1, 24, 24), (0, 0, 0), 50),       # two pair units per window, five routed tiles
+    (2, 2, 64, (3, 10, 13), (2, 4, 5), (1, 3, 2), 0),           # one-CTA kernel (d = 64)
+    (1, 2, 64, (2, 16, 16), (2, 8, 8), (0, 4, 4), 20),          # one-CTA kernel, full tiles plus memory
+])
+def test_fwd_route_matches_oracle(B, heads, d, grid, win, shift, E):
+    T, H, W = grid
+    q, k, v = make_custom(B, heads, d, T, H, W, seed=11 + E)
+    kx, vx = _extra(B, max(E, 1), heads, d, seed=2000 + E)
+    kx, vx = kx[:, :E].contiguous(), vx[:, :E].contiguous()
+    routed = _oracle_routes(q, k, B, heads, grid, d, win, shift)
+    scale = 1.0 / math.sqrt(d)
+    dev = torch.device("cuda:0")
+    rd = torch.from_numpy(routed).to(dev)
+    out = sw.swattn_fwd_route(q.to(dev), k.to(dev), v.to(dev), rd, grid, win, shift,
+                              kx.to(dev) if E else None, vx.to(dev) if E else None, scale)
+    assert sw.last_device_error() == sw.BASA_OK
+    ref = oracle.swattn_fwd_route(q, k, v, routed, kx if E else None, vx if E else None, E, B, heads, T, H, W,
+                                  d, win, shift, scale)
+    _check(out.float().cpu().numpy(), ref, f"routed E={E} grid={grid} win={win} d={d}")
+
+
+@pytest.mark.parametrize("d", [128, 64])
+def test_fwd_route_with_nothing_routed_is_bitwise_the_memory_forward(d):
+    grid, win, shift = (1, 24, 24), (1, 8, 8), (0, 4, 4)
+    q, k, v = make_custom(1, 2, d, *grid, seed=5)
+    kx, vx = _extra(1, 9, 2, d, seed=6)
+    dev = torch.device("cuda:0")
+    qd, kd, vd, kxd, vxd = (t.to(dev) for t in (q, k, v, kx, vx))
+    none = torch.full((1, 2, 9), -1, dtype=torch.int32, device=dev)
+    a = sw.swattn_fwd_route(qd, kd, vd, none, grid, win, shift, kxd, vxd)
+    b = sw.swattn_fwd_mem(qd, kd, vd, kxd, vxd, grid, win, shift)
+    c = sw.swattn_fwd_route(qd, kd, vd, none, grid, win, shift)
+    e = sw.swattn_fwd(qd, kd, vd, grid, win, shift)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b) and torch.equal(c, e)
+
+
+@pytest.mark.parametrize("d,grid,win,shift,pool", [
+    (128, (3, 20, 26), (3, 5, 6), (0, 2, 3), (1, 4, 4)),        # video: full temporal extent
+    (128, (1, 32, 32), (1, 8, 8), (0, 4, 4), (1, 4, 4)),        # image
+])
+def test_full_basa_pipeline(d, grid, win, shift, pool):
+    # S_i = W_i u R_i u G: GPU route, GPU pooling, GPU forward; the oracle runs its
+    # own routing and pooling (rounded to bf16 like every K/V operand) and forward
+    T, H, W = grid
+    B, heads = 1, 2
+    q, k, v = make_custom(B, heads, d, T, H, W, seed=8)
+    dev = torch.device("cuda:0")
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    rd = sw.route(qd, kd, grid, win, shift)
+    kbar, vbar = sw.kv_pool(kd, vd, grid, pool)
+    out = sw.swattn_fwd_route(qd, kd, vd, rd, grid, win, shift, kbar, vbar)
+    assert sw.last_device_error() == sw.BASA_OK
+    routed, scores = oracle.route(q, k, B, heads, T, H, W, d, win, shift, 1, with_scores=True)
+    dec, tot = _check_routes(rd.cpu().numpy(), routed, scores, "pipeline")
+    assert dec == tot, "this case is chosen so that every routing decision is clear"
+    G = oracle.n_pooled(T, H, W, pool)
+    kb = oracle.round_to_bf16_bits(oracle.kv_pool(k, B, heads, T, H, W, d, pool))
+    vb = oracle.round_to_bf16_bits(oracle.kv_pool(v, B, heads, T, H, W, d, pool))
+    ref = oracle.swattn_fwd_route(q, k, v, routed, kb, vb, G, B, heads, T, H, W, d, win, shift,
+                                  1.0 / math.sqrt(d))
+    _check(out.float().cpu().numpy(), ref, f"full BASA grid={grid}")
+
+
+@pytest.mark.parametrize("wl", [WORKLOADS[4], WORKLOADS[5]], ids=lambda w: w.name)
+def test_full_basa_full_size_sampled(wl):
+    # the launch configuration the benchmark's routing key times: routing, 1x4x4
+    # pooled memory and the routed forward, at full size; sampled rows
+    pool = (1, 4, 4)
+    q, k, v = make_qkv(wl)
+    shift = wl.shifts[-1]
+    dev = torch.device("cuda:0")
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    routed = oracle.route(q, k, wl.B, wl.heads, *wl.grid, wl.d, wl.win, shift, 1)
+    kbar, vbar = sw.kv_pool(kd, vd, wl.grid, pool)
+    out = sw.swattn_fwd_route(qd, kd, vd, torch.from_numpy(routed).to(dev), wl.grid, wl.win, shift, kbar, vbar,
+                              wl.scale)
+    assert sw.last_device_error() == sw.BASA_OK
+    G = oracle.n_pooled(*wl.grid, pool)
+    kb = oracle.round_to_bf16_bits(oracle.kv_pool(k, wl.B, wl.heads, *wl.grid, wl.d, pool))
+    vb = oracle.round_to_bf16_bits(oracle.kv_pool(v, wl.B, wl.heads, *wl.grid, wl.d, pool))
+    rng = np.random.default_rng(wl.seed + 50)
+    # random rows plus the first 300 queries of one window (three tiles, so the
+    # tile seams are covered; the oracle's cost per row grows with the key count)
+    tri = _sample_triples(wl, shift, 800, rng)
+    tri = tri[:800 + 300]
+    ref = oracle.swattn_rows_route(q, k, v, routed, kb, vb, G, wl.B, wl.heads, *wl.grid, wl.d, wl.win, shift,
+                                   wl.scale, tri)
+    got = out[tri[:, 0], tri[:, 1], tri[:, 2]].float().cpu().numpy()
+    _check(got, ref, f"{wl.name} full BASA")
+    assert torch.isfinite(out).all()
