@@ -503,3 +503,52 @@ def test_rows_route_agree_bitwise_with_full_routed_forward(E):
     triples = np.stack([rng.integers(0, B, 40), rng.integers(0, T * H * W, 40), rng.integers(0, heads, 40)], 1)
     rows = oracle.swattn_rows_route(*bits, routed, kx, vx, E, B, heads, T, H, W, d, win, shift, 0.4, triples)
     np.testing.assert_array_equal(rows, full[triples[:, 0], triples[:, 1], triples[:, 2]])
+
+
+def _branch(s, v):
+    """Softmax attention of one branch: (O, log-sum-exp) for logits s [n, m], values v [m, d]."""
+    mx = s.max(axis=1, keepdims=True)
+    e = np.exp(s - mx)
+    z = e.sum(axis=1, keepdims=True)
+    return (e / z) @ v, (mx + np.log(z))[:, 0]
+
+
+def test_single_softmax_equals_the_lse_merge_of_branches():
+    # Appendix A.1 runs the local window and the memory as separate attention calls and
+    # merges them with O = (1 - g) O_a + g O_b, g = sigmoid(l_b - l_a) (l = log-sum-exp);
+    # the kernels instead run one softmax over the concatenated keys.  The two agree:
+    # two-way {local} | {text + memory} and three-way {local} | {text} | {memory}
+    # merges, built branch by branch in numpy, reproduce the oracle's single softmax,
+    # and so does {local} | {routed} | {memory} for the routed forward (§3.3).
+    T, H, W, d, win, shift = 1, 8, 12, 8, (1, 4, 4), (0, 2, 1)
+    B, heads, E_txt, E_mem = 1, 2, 3, 5
+    bits, (q, k, v) = _qkv(B, heads, d, T, H, W, seed=31)
+    xbits, (kx, vx, _) = _qkv(B, heads, d, 1, 1, E_txt + E_mem, seed=32)
+    scale = 0.9 / math.sqrt(d)
+    wid = window_id_of_token(T, H, W, win, shift)
+    routed = oracle.route(bits[0], bits[1], B, heads, T, H, W, d, win, shift, 1)
+    single = oracle.swattn_fwd_mem(*bits, xbits[0], xbits[1], E_txt + E_mem, B, heads, T, H, W, d, win, shift,
+                                   scale)
+    single_rt = oracle.swattn_fwd_route(*bits, routed, xbits[0], xbits[1], E_txt + E_mem, B, heads, T, H, W, d,
+                                        win, shift, scale)
+
+    def merge(parts):
+        o, lse = parts[0]
+        for ob, lb in parts[1:]:
+            g = 1.0 / (1.0 + np.exp(-(lb - lse)))
+            o = (1.0 - g)[:, None] * o + g[:, None] * ob
+            lse = np.logaddexp(lse, lb)
+        return o
+
+    for h in range(heads):
+        qh, kh, vh = q[0, :, h], k[0, :, h], v[0, :, h]
+        s_loc = np.where(wid[:, None] == wid[None, :], scale * qh @ kh.T, -np.inf)
+        local = _branch(s_loc, vh)
+        txt = _branch(scale * qh @ kx[0, :E_txt, h].T, vx[0, :E_txt, h])
+        mem = _branch(scale * qh @ kx[0, E_txt:, h].T, vx[0, E_txt:, h])
+        both = _branch(scale * qh @ kx[0, :, h].T, vx[0, :, h])
+        np.testing.assert_allclose(merge([local, both]), single[0, :, h], rtol=0, atol=1e-13)
+        np.testing.assert_allclose(merge([local, txt, mem]), single[0, :, h], rtol=0, atol=1e-13)
+        rt = routed[0, h][wid]
+        s_rt = np.where(rt[:, None] == wid[None, :], scale * qh @ kh.T, -np.inf)
+        np.testing.assert_allclose(merge([local, _branch(s_rt, vh), both]), single_rt[0, :, h], rtol=0, atol=1e-13)
