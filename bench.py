@@ -48,11 +48,42 @@ KERNEL_SOURCES = ["shifted_window_attention_swattn_b200/csrc/swattn_sm100.cu",
                   "shifted_window_attention_swattn_b200/csrc/softmax_sm100.cuh"]
 
 
-def kernel_source_hash() -> str:
+def strip_c_comments(text: str) -> str:
+    """C/C++ source with its comments removed and runs of whitespace collapsed
+    (string and character literals kept as they are), so that editing a comment
+    does not change what the kernel hash identifies."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            out.append(" ")
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
+def kernel_source_hash(read=None) -> str:
+    """Hash of the kernel sources, comments and whitespace aside.  `read(rel)`
+    returns a file's text (default: the working tree)."""
+    if read is None:
+        def read(rel):
+            with open(os.path.join(ROOT, rel), encoding="utf-8") as f:
+                return f.read()
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        h.update(strip_c_comments(read(rel)).encode())
     return h.hexdigest()[:16]
 
 

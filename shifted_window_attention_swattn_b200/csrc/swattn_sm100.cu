@@ -30,6 +30,14 @@
 // TMEM columns: S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512); P_i is
 // bf16 over the front of S_i.
 //
+// Both kernels are templated on <kMem, kRoute>.  A unit's key tiles are those
+// of its window, then (kRoute, §3.3 "Content-Adaptive True-Window Routing")
+// those of its routed window, then (kMem, §3.2 "K/V-Pooled Global Memory")
+// those of an extra K/V segment such as the pooled memory; one online softmax
+// runs over all of them.  The routes come from win_desc_kernel (window means
+// of Q and K) and route_kernel (top-1 over the spatial neighbour windows), and
+// the pooled memory from kv_pool_kernel.
+//
 // Every mbarrier wait is bounded by a host-set timeout; a wait that runs out
 // raises a shared abort flag and a library-wide error word, every role stops
 // issuing work, the MMA issuer drains its in-flight MMAs, the producer drains
