@@ -219,3 +219,18 @@ def test_routing_entry_points_reject_bad_arguments_on_the_host(lib):
                                      shift, 0.1, None) == sw.BASA_ERR_ALIAS
     assert lib.basa_swattn_fwd_route(a, a, a, rt, None, None, 0, out, 1, 1, 1, 8, 8, 96, win, shift, 0.1,
                                      None) == sw.BASA_ERR_UNSUPPORTED
+
+
+def test_python_binding_routing_rejects_bad_tensors(lib):
+    import torch
+    q = torch.zeros(1, 16, 1, 64, dtype=torch.bfloat16)
+    with pytest.raises(TypeError):
+        sw.route(q, q, (1, 4, 4), (1, 2, 2), (0, 0, 0))
+    with pytest.raises(TypeError):
+        sw.route(q.float(), q.float(), (1, 4, 4), (1, 2, 2), (0, 0, 0))
+    routed = torch.zeros(1, 1, 4, dtype=torch.int32)
+    with pytest.raises((TypeError, ValueError)):
+        sw.swattn_fwd_route(q, q, q, routed, (1, 4, 4), (1, 2, 2), (0, 0, 0))
+    with pytest.raises(ValueError):
+        sw.n_windows((1, 4, 4), (1, 0, 2))
+    assert sw.n_windows((3, 10, 13), (2, 4, 5)) == oracle.n_windows(3, 10, 13, (2, 4, 5))
