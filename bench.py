@@ -372,6 +372,63 @@ def sweep_workloads(stream, flush, peak_tflops):
     return rows
 
 
+TARGET_WORKLOADS = {"flux4096": "flux-4096px-256x256-w32", "wan720p": "wan-720p-21x45x80-w7x15x16"}
+
+
+def targets_of(per_wl):
+    """Compact summary of the two workloads the stated targets (>= 0.55 of peak,
+    speedup >= 0.9 of N/n_w) apply to, from the per-workload table."""
+    out = {}
+    for key, name in TARGET_WORKLOADS.items():
+        rows = [r for r in per_wl if r["workload"] == name]
+        if not rows:
+            continue
+        r = rows[0]
+        out[key] = {"ms_window": [round(x["ms"], 4) for x in r["window"]],
+                    "tflops": round(r["flops_window"] / r["ms_window_mean"] / 1e9, 1),
+                    "frac_of_peak": round(statistics.mean(x["frac_of_peak"] for x in r["window"]), 4),
+                    "ms_full": round(r["ms_full"], 3), "full_frac_of_peak": round(r["full_frac_of_peak"], 4),
+                    "speedup_vs_full": round(r["speedup_vs_full"], 2),
+                    "speedup_frac_of_theoretical": round(r["speedup_frac_of_theoretical"], 4)}
+    return out
+
+
+def text_memory_case(stream, device, peak_tflops, n_text=512, pool=(1, 4, 4)):
+    """FLUX-like joint attention on the 4096^2 image grid: every visual query
+    attends to its window, n_text text tokens and the pooled memory of K and V
+    (one extra segment [text; pooled]).  Times the pooling and the forward."""
+    import torch
+    import shifted_window_attention_swattn_b200 as sw
+    from shifted_window_attention_swattn_b200.inputs import BY_NAME, make_custom, make_qkv
+    wl = BY_NAME[TARGET_WORKLOADS["flux4096"]]
+    q, k, v = make_qkv(wl, device=device)
+    kt, vt, _ = make_custom(wl.B, wl.heads, wl.d, 1, 1, n_text, seed=4343, device=device)
+    G = sw.kv_pool_tokens(wl.grid, pool)
+    kx = torch.empty((wl.B, n_text + G, wl.heads, wl.d), dtype=torch.bfloat16, device=device)
+    vx = torch.empty_like(kx)
+    kx[:, :n_text] = kt
+    vx[:, :n_text] = vt
+    out = torch.empty_like(q)
+    shift = wl.shifts[1]
+
+    def pool_step():
+        kbar, vbar = sw.kv_pool(k, v, wl.grid, pool, stream=stream)
+        kx[:, n_text:] = kbar
+        vx[:, n_text:] = vbar
+
+    def fwd():
+        sw.swattn_fwd_mem(q, k, v, kx, vx, wl.grid, wl.win, shift, wl.scale, out=out, stream=stream)
+    with torch.cuda.stream(stream):
+        pool_step()
+    time_launches(fwd, 3, stream)
+    ms_fwd = statistics.median(time_launches(fwd, 20, stream))
+    E = n_text + G
+    f_fwd = sw.flops(wl.B, wl.heads, wl.grid, wl.d, wl.win) + 4.0 * wl.B * wl.heads * wl.d * wl.N * E
+    return {"workload": wl.name, "shift_thw": list(shift), "text_tokens": n_text, "pool_thw": list(pool),
+            "pooled_tokens": G, "extra_tokens": E, "ms_fwd": ms_fwd, "flops_fwd": f_fwd,
+            "tflops_fwd": f_fwd / ms_fwd / 1e9, "frac_of_peak": f_fwd / ms_fwd / 1e9 / peak_tflops}
+
+
 def run_native(args):
     import torch
     import torch.distributed as dist
@@ -477,6 +534,8 @@ def run_native(args):
         flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
         per_wl = sweep_workloads(stream, flush, peak_tflops) if not args.no_sweep else []
         extras["per_workload"] = per_wl
+        if per_wl:
+            extras["targets"] = targets_of(per_wl)
         head = [r for r in per_wl if r["workload"] == wl.name]
         if head:
             extras["speedup_vs_full"] = head[0]["speedup_vs_full"]
@@ -563,6 +622,9 @@ def run_native(args):
                 "ms_fwd": ms_fwd_rt, "flops_fwd": f_rt, "tflops_fwd": f_rt / ms_fwd_rt / 1e9,
                 "source": "own window + routed window" + (" + pooled memory" if pool else "")}
             del ws, routed, kbar, vbar
+        if args.text_memory:
+            extras["text_memory"] = text_memory_case(stream, device, peak_tflops)
+            torch.cuda.empty_cache()
         # CPU baseline: the oracle on a bounded sample of the same workload
         if not args.no_cpu_baseline:
             qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
@@ -597,7 +659,14 @@ def run_native(args):
         "gpu_launches": launches,
         "clocks": clocks.summary(),
     }
+    # the compact target summary goes right after the configuration, the long
+    # per-workload table last
+    if "targets" in extras:
+        line = dict(list(line.items())[:13] + [("targets", extras.pop("targets"))] + list(line.items())[13:])
+    per_wl = extras.pop("per_workload", None)
     line.update(extras)
+    if per_wl is not None:
+        line["per_workload"] = per_wl
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -619,6 +688,9 @@ def main():
                     help="also time the pooled global memory: pooling factors t,h,w ('' to skip)")
     ap.add_argument("--route", action=argparse.BooleanOptionalAction, default=True,
                     help="time true-window routing and the routed forward (the `route` key)")
+    ap.add_argument("--text-memory", action=argparse.BooleanOptionalAction, default=True,
+                    help="time the FLUX-like joint attention: window + 512 text tokens + pooled memory "
+                         "(the `text_memory` key)")
     ap.add_argument("--schedule-layers", type=int, default=8,
                     help="also time an L-layer stack under the interleaved shift schedule (0: off)")
     ap.add_argument("--workload", default=HEADLINE,

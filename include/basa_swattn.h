@@ -161,6 +161,7 @@ int basa_route_workspace_bytes(int B, int heads, int T, int H, int W, int d, con
  * the same temporal window index whose (m_h, m_w) lie within Chebyshev
  * distance `radius` of i's, without wrap-around.  Ties go to the lower window
  * index; a window with no candidate (radius 0, or one spatial window) gets -1.
+ * A radius larger than the window grid is treated as the grid's extent.
  *
  *   q, k       device bf16 [B, T*H*W, heads, d], 16-byte aligned (as basa_swattn_fwd)
  *   workspace  device, >= basa_route_workspace_bytes(...) bytes, 16-byte
@@ -203,8 +204,9 @@ int basa_swattn_last_device_error(void* stream);
 
 /*
  * Upper bound, in nanoseconds, on every wait inside the kernels (default one
- * second).  A launch whose wait runs out stops its work, drains what it has in
- * flight, releases its tensor memory, and records BASA_ERR_DEVICE.
+ * second), process-wide: launches from every host thread read it.  A launch
+ * whose wait runs out stops its work, drains what it has in flight, releases
+ * its tensor memory, and records BASA_ERR_DEVICE.
  */
 int basa_swattn_set_wait_timeout_ns(unsigned long long ns);
 
@@ -212,7 +214,9 @@ int basa_swattn_set_wait_timeout_ns(unsigned long long ns);
  * Test hook for the bounded-wait error path (not part of the method): while
  * `on` is non-zero, every launch's MMA issuer first waits on a barrier that
  * nothing arrives on, so the launch times out after the wait limit, stops,
- * drains and reports BASA_ERR_DEVICE.  Off by default.
+ * drains and reports BASA_ERR_DEVICE.  Off by default.  The setting (like the
+ * wait limit above) is process-wide: it applies to launches made from every
+ * host thread while it is on.
  */
 int basa_swattn_set_test_stall(int on);
 

@@ -118,7 +118,27 @@ def _stream_handle(stream, device):
     import torch
     if stream is None:
         stream = torch.cuda.current_stream(device)
+    elif stream.device != device:
+        raise ValueError(f"stream is on {stream.device}, the tensors on {device}")
     return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _require_on(device, named):
+    """Every (name, tensor) pair holds a CUDA tensor on ``device``: the kernels
+    address all operands of a call on the GPU of its first input."""
+    import torch
+    for name, t in named:
+        if not isinstance(t, torch.Tensor) or not t.is_cuda or t.device != device:
+            where = t.device if isinstance(t, torch.Tensor) else type(t).__name__
+            raise ValueError(f"{name} must be a CUDA tensor on {device} (got {where})")
+
+
+def _call_on(device, fn, *args):
+    """Calls the C entry point with ``device`` current (the library launches on
+    the current device)."""
+    import torch
+    with torch.cuda.device(device):
+        return fn(*args)
 
 
 def swattn_fwd(q, k, v, grid, win, shift, scale=None, out=None, stream=None):
@@ -146,11 +166,11 @@ def swattn_fwd(q, k, v, grid, win, shift, scale=None, out=None, stream=None):
         out = torch.empty_like(q)
     elif out.shape != q.shape or out.dtype != torch.bfloat16 or not out.is_contiguous():
         raise ValueError("out must be a contiguous bf16 tensor shaped like q")
+    _require_on(q.device, (("k", k), ("v", v), ("out", out)))
     if scale is None:
         scale = d ** -0.5
-    rc = lib.basa_swattn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, heads,
-                             T, H, W, d, _I3(*w3), _I3(*s3), float(scale),
-                             _stream_handle(stream, q.device))
+    rc = _call_on(q.device, lib.basa_swattn_fwd, q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                  B, heads, T, H, W, d, _I3(*w3), _I3(*s3), float(scale), _stream_handle(stream, q.device))
     if rc != BASA_OK:
         raise SwattnError(rc, "basa_swattn_fwd")
     return out
@@ -180,12 +200,13 @@ def swattn_fwd_mem(q, k, v, kx, vx, grid, win, shift, scale=None, out=None, stre
         out = torch.empty_like(q)
     elif out.shape != q.shape or out.dtype != torch.bfloat16 or not out.is_contiguous():
         raise ValueError("out must be a contiguous bf16 tensor shaped like q")
+    _require_on(q.device, (("k", k), ("v", v), ("kx", kx), ("vx", vx), ("out", out)))
     if scale is None:
         scale = d ** -0.5
     E = kx.shape[1]
-    rc = lib.basa_swattn_fwd_mem(q.data_ptr(), k.data_ptr(), v.data_ptr(), kx.data_ptr(), vx.data_ptr(),
-                                 E, out.data_ptr(), B, heads, T, H, W, d, _I3(*w3), _I3(*s3),
-                                 float(scale), _stream_handle(stream, q.device))
+    rc = _call_on(q.device, lib.basa_swattn_fwd_mem, q.data_ptr(), k.data_ptr(), v.data_ptr(), kx.data_ptr(),
+                  vx.data_ptr(), E, out.data_ptr(), B, heads, T, H, W, d, _I3(*w3), _I3(*s3), float(scale),
+                  _stream_handle(stream, q.device))
     if rc != BASA_OK:
         raise SwattnError(rc, "basa_swattn_fwd_mem")
     return out
@@ -234,15 +255,17 @@ def route(q, k, grid, win, shift, radius=1, out=None, workspace=None, stream=Non
     need = route_workspace_bytes(B, heads, grid, d, win)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
-    elif not workspace.is_cuda or not workspace.is_contiguous():
+    elif not isinstance(workspace, torch.Tensor) or not workspace.is_contiguous():
         raise ValueError("workspace must be a contiguous CUDA tensor")
     if out is None:
         out = torch.empty((B, heads, nw), dtype=torch.int32, device=q.device)
     elif out.shape != (B, heads, nw) or out.dtype != torch.int32 or not out.is_contiguous():
         raise ValueError(f"out must be a contiguous int32 tensor of shape {(B, heads, nw)}")
+    _require_on(q.device, (("k", k), ("workspace", workspace), ("out", out)))
     ws_bytes = workspace.numel() * workspace.element_size()
-    rc = lib.basa_route(q.data_ptr(), k.data_ptr(), B, heads, T, H, W, d, _I3(*w3), _I3(*s3), int(radius),
-                        workspace.data_ptr(), ws_bytes, out.data_ptr(), _stream_handle(stream, q.device))
+    rc = _call_on(q.device, lib.basa_route, q.data_ptr(), k.data_ptr(), B, heads, T, H, W, d, _I3(*w3),
+                  _I3(*s3), int(radius), workspace.data_ptr(), ws_bytes, out.data_ptr(),
+                  _stream_handle(stream, q.device))
     if rc != BASA_OK:
         raise SwattnError(rc, "basa_route")
     return out
@@ -279,12 +302,15 @@ def swattn_fwd_route(q, k, v, routed, grid, win, shift, kx=None, vx=None, scale=
         out = torch.empty_like(q)
     elif out.shape != q.shape or out.dtype != torch.bfloat16 or not out.is_contiguous():
         raise ValueError("out must be a contiguous bf16 tensor shaped like q")
+    named = [("k", k), ("v", v), ("routed", routed), ("out", out)]
+    if E:
+        named += [("kx", kx), ("vx", vx)]
+    _require_on(q.device, named)
     if scale is None:
         scale = d ** -0.5
-    rc = lib.basa_swattn_fwd_route(q.data_ptr(), k.data_ptr(), v.data_ptr(), routed.data_ptr(),
-                                   kx.data_ptr() if E else None, vx.data_ptr() if E else None, E,
-                                   out.data_ptr(), B, heads, T, H, W, d, _I3(*w3), _I3(*s3), float(scale),
-                                   _stream_handle(stream, q.device))
+    rc = _call_on(q.device, lib.basa_swattn_fwd_route, q.data_ptr(), k.data_ptr(), v.data_ptr(), routed.data_ptr(),
+                  kx.data_ptr() if E else None, vx.data_ptr() if E else None, E, out.data_ptr(), B, heads,
+                  T, H, W, d, _I3(*w3), _I3(*s3), float(scale), _stream_handle(stream, q.device))
     if rc != BASA_OK:
         raise SwattnError(rc, "basa_swattn_fwd_route")
     return out
@@ -318,11 +344,12 @@ def kv_pool(k, v, grid, pool, stream=None):
     B, N, heads, d = k.shape
     if N != T * H * W:
         raise ValueError(f"token count {N} != T*H*W = {T * H * W}")
+    _require_on(k.device, (("v", v),))
     G = kv_pool_tokens(grid, p3)
     kbar = torch.empty((B, G, heads, d), dtype=torch.bfloat16, device=k.device)
     vbar = torch.empty_like(kbar)
-    rc = lib.basa_kv_pool(k.data_ptr(), v.data_ptr(), kbar.data_ptr(), vbar.data_ptr(), B, heads,
-                          T, H, W, d, _I3(*p3), _stream_handle(stream, k.device))
+    rc = _call_on(k.device, lib.basa_kv_pool, k.data_ptr(), v.data_ptr(), kbar.data_ptr(), vbar.data_ptr(), B,
+                  heads, T, H, W, d, _I3(*p3), _stream_handle(stream, k.device))
     if rc != BASA_OK:
         raise SwattnError(rc, "basa_kv_pool")
     return kbar, vbar
@@ -367,8 +394,8 @@ def index_map(grid, win, shift, device="cuda", stream=None):
     for n, w in zip((T, H, W), w3):
         nwin *= -(-n // w)
     out = torch.empty((nwin, w3[0] * w3[1] * w3[2]), dtype=torch.int32, device=device)
-    rc = lib.basa_swattn_index_map(T, H, W, _I3(*w3), _I3(*s3), out.data_ptr(),
-                                   _stream_handle(stream, out.device))
+    rc = _call_on(out.device, lib.basa_swattn_index_map, T, H, W, _I3(*w3), _I3(*s3), out.data_ptr(),
+                  _stream_handle(stream, out.device))
     if rc != BASA_OK:
         raise SwattnError(rc, "basa_swattn_index_map")
     return out

@@ -48,6 +48,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstddef>
 #include <math.h>
@@ -1286,8 +1287,9 @@ __global__ void index_map_kernel(Geometry g, int32_t* tos) {
 
 static std::mutex g_mutex;
 static PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
-static unsigned long long g_timeout_ns = 1000000000ull;
-static int g_stall = 0;   // test hook, see basa_swattn_set_test_stall
+// Read by every launch, written by the setters below from any host thread.
+static std::atomic<unsigned long long> g_timeout_ns{1000000000ull};
+static std::atomic<int> g_stall{0};   // test hook, see basa_swattn_set_test_stall
 constexpr int kMaxDevices = 64;
 static int g_dev_state[kMaxDevices];   // 0 unknown, 1 ready, negative error code
 
@@ -1481,8 +1483,8 @@ static int launch_fwd(const void* q, const void* k, const void* v, const int* ro
     pp.total_units = static_cast<int>(punits);
     pp.n_slots = pair_slots();
     pp.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
-    pp.timeout_ns = g_timeout_ns;
-    pp.stall = g_stall;
+    pp.timeout_ns = g_timeout_ns.load();
+    pp.stall = g_stall.load();
     const long long clusters = punits < g_pair_clusters[dev] ? punits : g_pair_clusters[dev];
     return launch_variant(swattn_fwd_pair_kernel<false, false>, swattn_fwd_pair_kernel<true, false>,
                           swattn_fwd_pair_kernel<false, true>, swattn_fwd_pair_kernel<true, true>, E > 0,
@@ -1508,8 +1510,8 @@ static int launch_fwd(const void* q, const void* k, const void* v, const int* ro
   p.total_units = static_cast<int>(units);
   p.n_slots = slots_for(d);
   p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
-  p.timeout_ns = g_timeout_ns;
-  p.stall = g_stall;
+  p.timeout_ns = g_timeout_ns.load();
+  p.stall = g_stall.load();
   // Persistent: one CTA per SM, each walking the units with a stride of the grid.
   const long long grid = units < g_sm_count[dev] ? units : g_sm_count[dev];
   return launch_variant(swattn_fwd_kernel<false, false>, swattn_fwd_kernel<true, false>,
@@ -1576,6 +1578,10 @@ extern "C" int basa_route(const void* q, const void* k, int B, int heads, int T,
       overlaps2(routed, rbytes, q, in_bytes) || overlaps2(routed, rbytes, k, in_bytes) ||
       overlaps2(routed, rbytes, workspace, need))
     return BASA_ERR_ALIAS;
+  // A radius past the window grid selects the same candidates as the grid's
+  // extent; clamping keeps the kernel's window arithmetic inside int.
+  const int rmax = g.nwin[1] > g.nwin[2] ? g.nwin[1] : g.nwin[2];
+  if (radius > rmax) radius = rmax;
   int dev = 0;
   rc = prepare_device(&dev);
   if (rc) return rc;
@@ -1748,14 +1754,12 @@ extern "C" int basa_swattn_last_device_error(void* stream) {
 }
 
 extern "C" int basa_swattn_set_wait_timeout_ns(unsigned long long ns) {
-  std::lock_guard<std::mutex> lock(g_mutex);
-  g_timeout_ns = ns;
+  g_timeout_ns.store(ns);
   return BASA_OK;
 }
 
 extern "C" int basa_swattn_set_test_stall(int on) {
-  std::lock_guard<std::mutex> lock(g_mutex);
-  g_stall = on ? 1 : 0;
+  g_stall.store(on ? 1 : 0);
   return BASA_OK;
 }
 

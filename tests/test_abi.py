@@ -131,6 +131,21 @@ def test_python_binding_rejects_non_cuda_tensors(lib):
         sw.swattn_fwd(q, q, q, (1, 4, 4), (1, 2, 2), (0, 0, 0))
 
 
+def test_python_binding_device_check_rejects_host_tensors():
+    # the check every entry point applies to its outputs, routes, workspace and
+    # extra segment: CUDA tensors on the first input's device, nothing else
+    import torch
+    dev = torch.device("cuda", 0)
+    cpu_out = torch.empty(1, 16, 1, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        sw._require_on(dev, (("out", cpu_out),))
+    with pytest.raises(ValueError):
+        sw._require_on(dev, (("routed", torch.zeros(1, 1, 4, dtype=torch.int32)),))
+    with pytest.raises(ValueError):
+        sw._require_on(dev, (("workspace", None),))
+    sw._require_on(dev, ())
+
+
 def test_shift_schedule_equals_oracle(lib):
     for L in (1, 2, 3, 5, 8, 19, 57):
         for win in ((1, 16, 16), (7, 15, 16), (7, 10, 13), (21, 1, 32), (3, 4, 300)):

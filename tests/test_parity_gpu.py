@@ -9,6 +9,8 @@ sampled rows that the oracle computes one by one, in the same launch
 configuration the benchmark times.
 """
 import math
+import os
+from concurrent.futures import ThreadPoolExecutor
 
 import numpy as np
 import pytest
@@ -16,7 +18,7 @@ import torch
 
 import oracle
 import shifted_window_attention_swattn_b200 as sw
-from shifted_window_attention_swattn_b200.inputs import WORKLOADS, make_custom, make_qkv
+from shifted_window_attention_swattn_b200.inputs import BY_NAME, WORKLOADS, make_custom, make_qkv
 
 pytestmark = pytest.mark.gpu
 
@@ -148,6 +150,24 @@ def test_host_buffer_entry_matches_device_entry():
     assert torch.equal(dev, host)
 
 
+def test_binding_rejects_operands_off_the_input_device():
+    # a CPU output (or routes, workspace, extra segment) next to CUDA inputs is
+    # refused before anything is launched
+    grid, win, shift = (1, 16, 16), (1, 8, 8), (0, 4, 4)
+    q, k, v = (t.cuda() for t in make_custom(1, 2, 128, *grid, seed=12))
+    with pytest.raises(ValueError):
+        sw.swattn_fwd(q, k, v, grid, win, shift, out=torch.empty(q.shape, dtype=torch.bfloat16))
+    with pytest.raises(ValueError):
+        sw.swattn_fwd_mem(q, k, v, k[:, :8].contiguous().cpu(), v[:, :8].contiguous(), grid, win, shift)
+    with pytest.raises(ValueError):
+        sw.route(q, k, grid, win, shift, out=torch.empty((1, 2, 4), dtype=torch.int32))
+    with pytest.raises(ValueError):
+        sw.route(q, k, grid, win, shift, workspace=torch.empty(1 << 16, dtype=torch.uint8))
+    with pytest.raises(ValueError):
+        sw.swattn_fwd_route(q, k, v, torch.full((1, 2, 4), -1, dtype=torch.int32), grid, win, shift)
+    torch.cuda.synchronize()
+
+
 # ---------------------------------------------------------------- full-size workloads, sampled rows
 
 def _sample_triples(wl, shift, n_random, rng):
@@ -192,6 +212,49 @@ def test_full_attention_mode_sampled(wl):
                              wl.scale, tri)
     got = out[tri[:, 0], tri[:, 1], tri[:, 2]].float().cpu().numpy()
     _check(got, ref, "full attention")
+
+
+def _oracle_rows_threaded(fn, tri, *args):
+    """fn(*args, triples) over chunks of `tri` on all host threads (the oracle's
+    per-row C path releases the GIL); rows in the order of `tri`."""
+    threads = max(1, len(os.sched_getaffinity(0)))
+    chunks = [c for c in np.array_split(tri, threads * 2) if len(c)]
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        parts = list(ex.map(lambda c: fn(*args, c), chunks))
+    return np.concatenate(parts)
+
+
+# The full-attention mode at the sizes the benchmark times it (the denominator of
+# the speedup over full attention): 65,536 to 131,040 keys per query, 512 to 1,024
+# key steps per 512-query unit.  Random rows of every head, plus every query of
+# the last 512-query unit of one head (ragged on two of the grids), so that whole
+# long key loops, including the tail unit, are checked against fp64.
+FULL_MODE_AT_BENCH_SIZE = [BY_NAME["flux-4096px-256x256-w32"], BY_NAME["wan-720p-21x45x80-w7x15x16"],
+                           BY_NAME["wan-pages-21x60x104-w21x15x26"]]
+
+
+@pytest.mark.parametrize("wl", FULL_MODE_AT_BENCH_SIZE, ids=lambda w: w.name)
+def test_full_attention_mode_at_benchmark_size_sampled(wl):
+    q, k, v = make_qkv(wl)
+    dev = torch.device("cuda:0")
+    out = sw.swattn_fwd(q.to(dev), k.to(dev), v.to(dev), wl.grid, wl.grid, (0, 0, 0), wl.scale)
+    assert sw.last_device_error() == sw.BASA_OK
+    rng = np.random.default_rng(wl.seed + 700)
+    n_rand = 400
+    tri = np.stack([rng.integers(0, wl.B, n_rand), rng.integers(0, wl.N, n_rand),
+                    rng.integers(0, wl.heads, n_rand)], axis=1)
+    q0 = ((wl.N - 1) // 512) * 512                      # first query of the last unit
+    toks = np.arange(q0, wl.N)
+    head = int(rng.integers(0, wl.heads))
+    unit = np.stack([np.zeros_like(toks), toks, np.full_like(toks, head)], axis=1)
+    tri = np.concatenate([tri, unit]).astype(np.int64)
+    qb, kb, vb = oracle._bits(q), oracle._bits(k), oracle._bits(v)
+    ref = _oracle_rows_threaded(oracle.swattn_rows, tri, qb, kb, vb, wl.B, wl.heads, *wl.grid, wl.d, wl.grid,
+                                (0, 0, 0), wl.scale)
+    got = out[tri[:, 0], tri[:, 1], tri[:, 2]].float().cpu().numpy()
+    _check(got[:n_rand], ref[:n_rand], f"{wl.name} full attention, random rows")
+    _check(got[n_rand:], ref[n_rand:], f"{wl.name} full attention, last unit of head {head}")
+    assert torch.isfinite(out).all()
 
 
 @pytest.mark.parametrize("d,grid,win,L", [
@@ -286,6 +349,70 @@ def test_pooled_memory_pipeline(d, grid, win, shift, pool):
     _check(out.float().cpu().numpy(), ref, f"pooled memory grid={grid} pool={pool}")
 
 
+def _text_plus_memory(kd, vd, grid, pool, n_text, seed):
+    """The extra segment of the FLUX-like joint attention: n_text text tokens
+    (seeded N(0,1) bf16, [B, n_text, heads, d]) followed by the pooled memory
+    of K and V; returns the GPU tensors and the oracle's copy of the segment
+    (text bits as drawn, pooled tokens from the oracle's own pooling rounded to
+    bf16)."""
+    B, _, heads, d = kd.shape
+    kt, vt, _ = make_custom(B, heads, d, 1, 1, n_text, seed=seed)
+    kbar, vbar = sw.kv_pool(kd, vd, grid, pool)
+    kx = torch.cat([kt.to(kd.device), kbar], dim=1).contiguous()
+    vx = torch.cat([vt.to(kd.device), vbar], dim=1).contiguous()
+    return kx, vx, kt, vt
+
+
+def _oracle_segment(t, x, B, heads, grid, d, pool):
+    """Text bits followed by the oracle's pooled memory of x, as uint16 bf16 bits."""
+    pooled = oracle.round_to_bf16_bits(oracle.kv_pool(x, B, heads, *grid, d, pool))
+    return np.ascontiguousarray(np.concatenate([oracle._bits(t), pooled], axis=1))
+
+
+def test_text_and_pooled_memory_flux1024_every_element():
+    # visual queries of FLUX-1024 attend to their window, 512 text tokens and the
+    # 1x4x4 pooled memory (256 tokens), in one softmax
+    wl = BY_NAME["flux-1024px-64x64-w16"]
+    pool, n_text = (1, 4, 4), 512
+    q, k, v = make_qkv(wl)
+    dev = torch.device("cuda:0")
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    kx, vx, kt, vt = _text_plus_memory(kd, vd, wl.grid, pool, n_text, seed=4242)
+    E = kx.shape[1]
+    assert E == n_text + oracle.n_pooled(*wl.grid, pool)
+    shift = wl.shifts[1]
+    out = sw.swattn_fwd_mem(qd, kd, vd, kx, vx, wl.grid, wl.win, shift, wl.scale)
+    assert sw.last_device_error() == sw.BASA_OK
+    kxs = _oracle_segment(kt, k, wl.B, wl.heads, wl.grid, wl.d, pool)
+    vxs = _oracle_segment(vt, v, wl.B, wl.heads, wl.grid, wl.d, pool)
+    ref = oracle.swattn_fwd_mem(q, k, v, kxs, vxs, E, wl.B, wl.heads, *wl.grid, wl.d, wl.win, shift, wl.scale)
+    _check(out.float().cpu().numpy(), ref, "FLUX-1024 text + pooled memory")
+
+
+def test_text_and_pooled_memory_flux4096_sampled():
+    # the benchmark's text_memory configuration: FLUX-4096, 512 text tokens plus the
+    # 1x4x4 pooled memory (4,096 tokens); sampled rows, one whole window included
+    wl = BY_NAME["flux-4096px-256x256-w32"]
+    pool, n_text = (1, 4, 4), 512
+    q, k, v = make_qkv(wl)
+    dev = torch.device("cuda:0")
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    kx, vx, kt, vt = _text_plus_memory(kd, vd, wl.grid, pool, n_text, seed=4343)
+    E = kx.shape[1]
+    shift = wl.shifts[1]
+    out = sw.swattn_fwd_mem(qd, kd, vd, kx, vx, wl.grid, wl.win, shift, wl.scale)
+    assert sw.last_device_error() == sw.BASA_OK
+    kxs = _oracle_segment(kt, k, wl.B, wl.heads, wl.grid, wl.d, pool)
+    vxs = _oracle_segment(vt, v, wl.B, wl.heads, wl.grid, wl.d, pool)
+    rng = np.random.default_rng(77)
+    tri = _sample_triples(wl, shift, 600, rng)
+    none = np.full((wl.B, wl.heads, sw.n_windows(wl.grid, wl.win)), -1, dtype=np.int32)
+    ref = _oracle_rows_threaded(oracle.swattn_rows_route, tri, oracle._bits(q), oracle._bits(k), oracle._bits(v),
+                                none, kxs, vxs, E, wl.B, wl.heads, *wl.grid, wl.d, wl.win, shift, wl.scale)
+    got = out[tri[:, 0], tri[:, 1], tri[:, 2]].float().cpu().numpy()
+    _check(got, ref, "FLUX-4096 text + pooled memory")
+
+
 # ---------------------------------------------------------------- true-window routing (§3.3)
 
 ROUTE_TAU = 1e-4   # score margin, relative to the row's largest |s_ij|, inside which fp32 may pick either
@@ -336,6 +463,18 @@ def test_route_is_deterministic():
     a = sw.route(qd, kd, grid, win, shift)
     for _ in range(3):
         assert torch.equal(a, sw.route(qd, kd, grid, win, shift))
+
+
+def test_route_radius_beyond_the_window_grid():
+    # a radius past the window grid (up to INT_MAX) selects every spatial neighbour
+    grid, win, shift = (2, 20, 26), (1, 5, 6), (1, 2, 3)
+    q, k, _ = make_custom(1, 2, 128, *grid, seed=31)
+    qd, kd = q.cuda(), k.cuda()
+    a = sw.route(qd, kd, grid, win, shift, radius=5)             # covers the 4 x 5 window grid
+    for big in (6, 1000, 2 ** 31 - 1):
+        assert torch.equal(a, sw.route(qd, kd, grid, win, shift, radius=big)), big
+    ref, scores = oracle.route(q, k, 1, 2, *grid, 128, win, shift, 5, with_scores=True)
+    _check_routes(a.cpu().numpy(), ref, scores, "radius covering the grid")
 
 
 @pytest.mark.parametrize("wl", WORKLOADS[1:], ids=lambda w: w.name)
