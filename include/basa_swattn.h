@@ -48,6 +48,7 @@ extern "C" {
 #define BASA_ERR_CUDA (-4)         /* a CUDA runtime or driver call failed */
 #define BASA_ERR_DEVICE (-5)       /* a bounded device-side wait expired in a launch */
 #define BASA_ERR_ALIAS (-6)        /* out overlaps q, k or v */
+#define BASA_ERR_SCRATCH_LIMIT (-7) /* larger than the fixed device scratch of basa_route_noalloc */
 
 /*
  * Shifted-window attention forward (§3.1 "Shifted Window Sparse Attention").
@@ -178,6 +179,39 @@ int basa_route_workspace_bytes(int B, int heads, int T, int H, int W, int d, con
 int basa_route(const void* q, const void* k, int B, int heads, int T, int H, int W, int d,
                const int win[3], const int shift[3], int radius, void* workspace,
                size_t workspace_bytes, int32_t* routed, void* stream);
+
+/*
+ * Bytes of device scratch basa_route_noalloc has: a fixed array inside the
+ * library, 4 MiB.
+ */
+#define BASA_ROUTE_NOALLOC_SCRATCH_BYTES (4u << 20)
+
+/*
+ * basa_route without a workspace argument, for callers that cannot allocate
+ * device memory at the point where they route: code running inside another
+ * framework's execution step (a plugin's enqueue callback, a serving loop that
+ * owns a fixed memory budget) where cudaMalloc is forbidden or would stall the
+ * device.  The paper has no counterpart; this is a deployment variant of the
+ * routing above.
+ *
+ * Same arguments, results, errors and ownership as basa_route, minus the
+ * workspace: the window descriptors (2 * B * heads * n_windows * d * 4 bytes)
+ * are kept in a fixed array of BASA_ROUTE_NOALLOC_SCRATCH_BYTES bytes inside
+ * the library, which every GPU that loads the library holds until the process
+ * exits.  A problem whose descriptors do not fit returns
+ * BASA_ERR_SCRATCH_LIMIT before anything is launched (B * heads * n_windows *
+ * d up to 524,288: e.g. 4,096 window-heads at d = 128).  The call allocates
+ * nothing and calls no allocating routine.
+ *
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  All calls on a device share the one array:
+ * calls whose work can overlap on the GPU (on different streams, or from
+ * different host threads without ordering) race on it and must not be made.
+ * Each call overwrites every descriptor it reads, so no clearing is needed.
+ */
+int basa_route_noalloc(const void* q, const void* k, int B, int heads, int T, int H, int W, int d,
+                       const int win[3], const int shift[3], int radius, int32_t* routed, void* stream);
 
 /*
  * The forward over the key/value source S_i = W_i u R_i u G of §3.3: the

@@ -18,7 +18,7 @@ import threading
 __all__ = [
     "swattn_fwd", "swattn_fwd_from_host", "swattn_fwd_mem", "kv_pool", "kv_pool_tokens",
     "index_map", "index_map_host", "flops", "shift_schedule", "route", "route_workspace_bytes",
-    "swattn_fwd_route", "n_windows",
+    "swattn_fwd_route", "route_noalloc", "n_windows",
     "last_device_error", "set_wait_timeout_ns", "strerror", "library_path", "SwattnError",
 ]
 
@@ -35,6 +35,8 @@ BASA_ERR_ALIGNMENT = -3
 BASA_ERR_CUDA = -4
 BASA_ERR_DEVICE = -5
 BASA_ERR_ALIAS = -6
+BASA_ERR_SCRATCH_LIMIT = -7
+ROUTE_NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
 class SwattnError(RuntimeError):
@@ -79,6 +81,8 @@ def _load():
         lib.basa_route_workspace_bytes.restype = ci
         lib.basa_route.argtypes = [vp, vp] + [ci] * 6 + [_I3, _I3, ci, vp, ctypes.c_size_t, vp, vp]
         lib.basa_route.restype = ci
+        lib.basa_route_noalloc.argtypes = [vp, vp] + [ci] * 6 + [_I3, _I3, ci, vp, vp]
+        lib.basa_route_noalloc.restype = ci
         lib.basa_swattn_fwd_route.argtypes = [vp] * 6 + [ci, vp] + [ci] * 6 + [_I3, _I3, ctypes.c_float, vp]
         lib.basa_swattn_fwd_route.restype = ci
         lib.basa_swattn_last_device_error.argtypes = [vp]
@@ -268,6 +272,33 @@ def route(q, k, grid, win, shift, radius=1, out=None, workspace=None, stream=Non
                   _stream_handle(stream, q.device))
     if rc != BASA_OK:
         raise SwattnError(rc, "basa_route")
+    return out
+
+
+def route_noalloc(q, k, grid, win, shift, radius=1, out=None, stream=None):
+    """``route`` through basa_route_noalloc: the library keeps the window
+    descriptors in its own fixed device array, so the C call allocates nothing
+    (for callers that cannot allocate at routing time).  Problems whose
+    descriptors exceed ROUTE_NOALLOC_SCRATCH_BYTES raise SwattnError
+    (BASA_ERR_SCRATCH_LIMIT).  Calls that can overlap on the GPU race on the
+    shared array.  ``out`` (int32 [B, heads, n_windows]) is allocated here when
+    not given."""
+    import torch
+    lib = _load()
+    T, H, W = _triple(grid, "grid")
+    w3, s3 = _triple(win, "win"), _triple(shift, "shift")
+    _check_qkv((("q", q), ("k", k)), (T, H, W))
+    B, _, heads, d = q.shape
+    nw = n_windows(grid, win)
+    if out is None:
+        out = torch.empty((B, heads, nw), dtype=torch.int32, device=q.device)
+    elif out.shape != (B, heads, nw) or out.dtype != torch.int32 or not out.is_contiguous():
+        raise ValueError(f"out must be a contiguous int32 tensor of shape {(B, heads, nw)}")
+    _require_on(q.device, (("k", k), ("out", out)))
+    rc = _call_on(q.device, lib.basa_route_noalloc, q.data_ptr(), k.data_ptr(), B, heads, T, H, W, d, _I3(*w3),
+                  _I3(*s3), int(radius), out.data_ptr(), _stream_handle(stream, q.device))
+    if rc != BASA_OK:
+        raise SwattnError(rc, "basa_route_noalloc")
     return out
 
 

@@ -1608,6 +1608,84 @@ extern "C" int basa_route(const void* q, const void* k, int B, int heads, int T,
   return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;
 }
 
+// ------------------------------------------------------------------ routing without allocation
+//
+// basa_route_noalloc is basa_route for callers that cannot allocate device
+// memory: code running inside another framework's execution step (a plugin's
+// enqueue, a serving loop with a fixed memory budget) where cudaMalloc is
+// forbidden or would stall the device.  Its window descriptors live in this
+// file-scope array instead of a caller's workspace.  Every GPU that loads the
+// library holds the array until the process exits, and every call on a device
+// shares it: calls whose work overlaps on the GPU (two streams, or two host
+// threads) race on it.  Each call overwrites every descriptor it reads, so
+// nothing needs clearing between calls.
+constexpr size_t kRouteScratchBytes = BASA_ROUTE_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) unsigned char g_route_scratch[kRouteScratchBytes];
+// Device address of g_route_scratch on each device (host code cannot use the
+// array's name as a device address), found on the first call on that device.
+static void* g_route_scratch_addr[kMaxDevices];
+
+static int route_scratch_address(int dev, void** addr) {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (!g_route_scratch_addr[dev]) {
+    void* a = nullptr;
+    if (cudaGetSymbolAddress(&a, g_route_scratch) != cudaSuccess || !a) return BASA_ERR_CUDA;
+    g_route_scratch_addr[dev] = a;
+  }
+  *addr = g_route_scratch_addr[dev];
+  return BASA_OK;
+}
+
+extern "C" int basa_route_noalloc(const void* q, const void* k, int B, int heads, int T, int H, int W, int d,
+                                  const int win[3], const int shift[3], int radius, int32_t* routed,
+                                  void* stream) {
+  if (!q || !k || !routed || B < 1 || heads < 1 || radius < 0) return BASA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return BASA_ERR_UNSUPPORTED;
+  Geometry g;
+  int rc = make_geometry(&g, T, H, W, win, shift);
+  if (rc) return rc;
+  const long long rows = static_cast<long long>(B) * g.N * heads;
+  const long long descs = static_cast<long long>(B) * heads * g.n_windows;
+  if (rows >= (1LL << 31) || descs >= (1LL << 31)) return BASA_ERR_UNSUPPORTED;
+  // two fp32 descriptor arrays (window means of Q and of K)
+  if (static_cast<unsigned long long>(descs) * d * 2 * sizeof(float) > kRouteScratchBytes)
+    return BASA_ERR_SCRATCH_LIMIT;
+  if ((reinterpret_cast<uintptr_t>(q) & 15) || (reinterpret_cast<uintptr_t>(k) & 15)) return BASA_ERR_ALIGNMENT;
+  if (reinterpret_cast<uintptr_t>(routed) & 3) return BASA_ERR_ALIGNMENT;
+  const size_t in_bytes = static_cast<size_t>(rows) * d * 2;
+  const size_t rbytes = static_cast<size_t>(descs) * sizeof(int32_t);
+  if (overlaps2(routed, rbytes, q, in_bytes) || overlaps2(routed, rbytes, k, in_bytes)) return BASA_ERR_ALIAS;
+  const int rmax = g.nwin[1] > g.nwin[2] ? g.nwin[1] : g.nwin[2];
+  if (radius > rmax) radius = rmax;
+  int dev = 0;
+  rc = prepare_device(&dev);
+  if (rc) return rc;
+  void* scratch = nullptr;
+  rc = route_scratch_address(dev, &scratch);
+  if (rc) return rc;
+  DescParams dp;
+  dp.q = static_cast<const __nv_bfloat16*>(q);
+  dp.k = static_cast<const __nv_bfloat16*>(k);
+  dp.qbar = static_cast<float*>(scratch);
+  dp.kbar = dp.qbar + descs * d;
+  dp.g = g;
+  dp.B = B;
+  dp.heads = heads;
+  dp.d = d;
+  win_desc_kernel<<<static_cast<unsigned>(descs), kDescThreads, 0, static_cast<cudaStream_t>(stream)>>>(dp);
+  RouteParams rp;
+  rp.qbar = dp.qbar;
+  rp.kbar = dp.kbar;
+  rp.routed = routed;
+  rp.g = g;
+  rp.total = descs;
+  rp.d = d;
+  rp.radius = radius;
+  const long long blocks = (descs * 32 + 255) / 256;
+  route_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(rp);
+  return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;
+}
+
 extern "C" int basa_swattn_index_map(int T, int H, int W, const int win[3], const int shift[3],
                                      int32_t* d_token_of_slot, void* stream) {
   if (!d_token_of_slot) return BASA_ERR_INVALID_ARG;
@@ -1772,6 +1850,7 @@ extern "C" const char* basa_strerror(int code) {
     case BASA_ERR_CUDA: return "CUDA call failed";
     case BASA_ERR_DEVICE: return "a device-side wait timed out";
     case BASA_ERR_ALIAS: return "out overlaps an input";
+    case BASA_ERR_SCRATCH_LIMIT: return "problem needs more than the library's fixed device scratch";
     default: return "unknown error";
   }
 }
