@@ -76,6 +76,10 @@ WORKLOADS = (
              ((0, 0, 0), (0, 7, 13)), 5),
     Workload("wan-pages-21x60x104-w21x10x10", 1, 12, 128, 21, 60, 104, (21, 10, 10),
              ((0, 0, 0), (0, 5, 5)), 6),
+    # Head dimension 64 at scale (the 16x16 small case grown to a 256x256 grid
+    # with 24 heads): half the MMA work per exponential of the d = 128
+    # workloads, so the softmax's exponentials weigh twice as much.
+    Workload("d64-256x256-w16", 1, 24, 64, 1, 256, 256, (1, 16, 16), ((0, 0, 0), (0, 8, 8)), 7),
 )
 
 BY_NAME = {w.name: w for w in WORKLOADS}
