@@ -1,6 +1,7 @@
 // ptx_sm100.cuh -- thin inline-PTX wrappers for the sm_100a features the
-// shifted-window attention kernel uses: mbarriers, TMA tile::gather4 loads,
-// tcgen05 (TMEM allocation, UMMA issue/commit, TMEM loads/stores) and fences.
+// shifted-window attention kernel uses: mbarriers, TMA tile::gather4 loads and
+// tile::scatter4 stores (bulk async-groups), tcgen05 (TMEM allocation, UMMA
+// issue/commit, TMEM loads/stores) and fences.
 //
 // Encodings follow the PTX ISA (tcgen05 instruction and shared-memory matrix
 // descriptors).  No cluster multicast form of any load is used anywhere.
@@ -185,6 +186,38 @@ __device__ __forceinline__ void tma_gather4_pair(const CUtensorMap* map, uint32_
       "l"(reinterpret_cast<uint64_t>(map)), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3),
       "r"(bar_cluster)
       : "memory");
+}
+
+// Four rows (r0..r3) of a 2D tensor map whose box is {cols, 1}, stored from
+// 4 * cols * elem_bytes bytes at smem_src (laid out and swizzled as a load
+// through the same map would leave them); joins this thread's bulk async-group.
+__device__ __forceinline__ void tma_scatter4(const CUtensorMap* map, const void* smem_src, int32_t col,
+                                             int32_t r0, int32_t r1, int32_t r2, int32_t r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.tile::scatter4.bulk_group [%0, {%1, %2, %3, %4, %5}], [%6];"
+      ::"l"(reinterpret_cast<uint64_t>(map)), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3),
+      "r"(smem_u32(smem_src))
+      : "memory");
+}
+
+// Closes this thread's current bulk async-group.
+__device__ __forceinline__ void bulk_commit_group() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// Every bulk store of this thread has finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_group_read0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+// Every bulk store of this thread is complete.
+__device__ __forceinline__ void bulk_wait_group0() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
+__device__ __forceinline__ void st_shared_v4(void* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(p)), "r"(a), "r"(b), "r"(c), "r"(d)
+               : "memory");
 }
 
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {

@@ -18,12 +18,16 @@
 //     with the max kept stale until it grows by more than 2^8 so that O is
 //     rarely rescaled;
 //   * the inverse roll is the row address of the output store: each query's
-//     result is written back to the token row it was gathered from.
+//     result is written back to the token row it was gathered from (in the
+//     CTA-pair kernel by tile::scatter4 TMA stores from a staging tile, four
+//     rows per store, while the softmax warps go on to the next unit).
 //
 // Two persistent kernels share this pipeline.  A work unit is a run of query
 // tiles of one window of one (batch, head); each unit streams the window's
 // K/V tiles through a shared-memory ring, and two query tiles per CTA are
 // processed in ping-pong (softmax of one tile overlaps the MMAs of the other).
+// Unit and slot decoding divide by launch constants through precomputed
+// multiply-shift reciprocals (FastDiv), not integer division.
 //   * swattn_fwd_pair_kernel (d = 128): clusters of two CTAs issue M = 256
 //     MMAs with cta_group::2; each SM loads half of every K/V tile;
 //   * swattn_fwd_kernel (any supported d, one CTA per SM): M = 128 MMAs.
@@ -78,6 +82,28 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units: O is rescaled when the
 
 // ------------------------------------------------------------------ geometry
 
+// Division of 0 <= n < 2^31 by a divisor 1 <= d < 2^31 fixed for a launch, as
+// a multiply and a shift: with p = 31 + ceil(log2 d) and m = ceil(2^p / d),
+// floor(n * m / 2^p) = floor(n / d), because m * d - 2^p < d makes the error
+// term n (m d - 2^p) / (d 2^p) smaller than 1/d.  m < 2^32.
+struct FastDiv {
+  uint32_t d, m, p;
+};
+
+static inline FastDiv make_fastdiv(int d) {
+  FastDiv f;
+  uint32_t l = 0;
+  while ((1ull << l) < static_cast<unsigned long long>(d)) ++l;
+  f.d = static_cast<uint32_t>(d);
+  f.p = 31 + l;
+  f.m = static_cast<uint32_t>(((1ull << f.p) + static_cast<unsigned long long>(d) - 1) / static_cast<unsigned long long>(d));
+  return f;
+}
+
+__host__ __device__ __forceinline__ int fdiv(int n, const FastDiv& f) {
+  return static_cast<int>((static_cast<unsigned long long>(static_cast<uint32_t>(n)) * f.m) >> f.p);
+}
+
 // Grid, window and shift of one call.  Shared by the kernel, the index-map
 // kernel and the host index map, so that all three agree bit for bit.
 struct Geometry {
@@ -88,15 +114,23 @@ struct Geometry {
   int n_windows;  // product of nwin
   int nw_max;     // w_t * w_h * w_w
   int N;          // T * H * W
+  FastDiv f_nwin[3];   // by nwin[a]
+  FastDiv f_w[3];      // by w[a]: a full window's extent
+  FastDiv f_tail[3];   // by the extent of the last window along a (n_a - (nwin_a - 1) w_a)
 };
+
+// Division by e, the extent along axis a of one of the windows of g.
+__host__ __device__ __forceinline__ int div_extent(const Geometry& g, int a, int n, int e) {
+  return fdiv(n, e == g.w[a] ? g.f_w[a] : g.f_tail[a]);
+}
 
 // Window coordinates m and extents e (truncated at the grid edge) of window `id`
 // (raster order over m_t, m_h, m_w).
 __host__ __device__ __forceinline__ void window_of(const Geometry& g, int id, int m[3], int e[3]) {
-  m[2] = id % g.nwin[2];
-  const int r = id / g.nwin[2];
-  m[1] = r % g.nwin[1];
-  m[0] = r / g.nwin[1];
+  const int r = fdiv(id, g.f_nwin[2]);
+  m[2] = id - r * g.nwin[2];
+  m[0] = fdiv(r, g.f_nwin[1]);
+  m[1] = r - m[0] * g.nwin[1];
 #pragma unroll
   for (int a = 0; a < 3; ++a) {
     const int left = g.n[a] - m[a] * g.w[a];
@@ -109,10 +143,10 @@ __host__ __device__ __forceinline__ void window_of(const Geometry& g, int id, in
 // coordinate m_a*w_a + s_a holds original coordinate (m_a*w_a + s_a + Delta_a) mod n_a.
 __host__ __device__ __forceinline__ int slot_token(const Geometry& g, const int m[3],
                                                    const int e[3], int s) {
-  const int sw = s % e[2];
-  const int r = s / e[2];
-  const int sh = r % e[1];
-  const int st = r / e[1];
+  const int r = div_extent(g, 2, s, e[2]);
+  const int sw = s - r * e[2];
+  const int st = div_extent(g, 1, r, e[1]);
+  const int sh = r - st * e[1];
   int pt = m[0] * g.w[0] + st + g.delta[0];
   int ph = m[1] * g.w[1] + sh + g.delta[1];
   int pw = m[2] * g.w[2] + sw + g.delta[2];
@@ -135,6 +169,9 @@ static int make_geometry(Geometry* g, int T, int H, int W, const int win[3], con
     if (s < 0) s += g->n[a];
     g->delta[a] = static_cast<int>(s);
     g->nwin[a] = (g->n[a] + win[a] - 1) / win[a];
+    g->f_nwin[a] = make_fastdiv(g->nwin[a]);
+    g->f_w[a] = make_fastdiv(win[a]);
+    g->f_tail[a] = make_fastdiv(g->n[a] - (g->nwin[a] - 1) * win[a]);
     N *= g->n[a];
     nwin *= g->nwin[a];
     nmax *= win[a];
@@ -157,6 +194,7 @@ struct __align__(64) FwdParams {
   Geometry g;
   int B, heads, d;
   int q_pairs;                  // ceil(nw_max / 256): 256-query units per window
+  FastDiv f_qp, f_nw, f_heads;  // by q_pairs, n_windows, heads
   int total_units;              // B * heads * n_windows * q_pairs
   int n_slots;                  // K/V ring depth (tiles)
   float scale_log2;             // scale * log2(e)
@@ -235,11 +273,11 @@ __device__ __forceinline__ void route_of(const Geometry& g, const int* routed, i
 // (batch, head), so CTAs that run at the same time share K/V in L2.
 template <bool kMem, bool kRoute>
 __device__ __forceinline__ bool decode_unit(const FwdParams& p, int u, Unit& U) {
-  const int qp = u % p.q_pairs;
-  const int r = u / p.q_pairs;
-  const int win_id = r % p.g.n_windows;
-  const int bh = r / p.g.n_windows;
-  U.b = bh / p.heads;
+  const int r = fdiv(u, p.f_qp);
+  const int qp = u - r * p.q_pairs;
+  const int bh = fdiv(r, p.f_nw);
+  const int win_id = r - bh * p.g.n_windows;
+  U.b = fdiv(bh, p.f_heads);
   U.h = bh - U.b * p.heads;
   window_of(p.g, win_id, U.m, U.e);
   U.n_valid = U.e[0] * U.e[1] * U.e[2];
@@ -309,10 +347,10 @@ __device__ __forceinline__ void extra_rows4(const Unit& U, int heads, int s, int
 // raster order.
 __device__ __forceinline__ void win_rows4(const Geometry& g, int b, int h, const int m[3], const int e[3],
                                           int heads, int s, int r[4]) {
-  int sw = s % e[2];
-  const int q = s / e[2];
-  int sh = q % e[1];
-  int st = q / e[1];
+  const int q = div_extent(g, 2, s, e[2]);
+  int sw = s - q * e[2];
+  int st = div_extent(g, 1, q, e[1]);
+  int sh = q - st * e[1];
   const int base_t = m[0] * g.w[0] + g.delta[0];
   const int base_h = m[1] * g.w[1] + g.delta[1];
   const int base_w = m[2] * g.w[2] + g.delta[2];
@@ -715,12 +753,14 @@ constexpr int kPairMaxSlots = 12;
 struct __align__(64) PairParams {
   CUtensorMap tq, tk, tv;       // 2D [rows = B*N*heads, cols = 128], box {64, 1}, 128B swizzle
   CUtensorMap tkx, tvx;         // extra K/V segment, 2D [rows = B*n_extra*heads, cols = 128] (kMem)
+  CUtensorMap to;               // the output, same view as tq (tile::scatter4 stores of the epilogue)
   int n_extra;                  // extra keys appended to every window (kMem)
   const int* routed;            // [B, heads, n_windows] routed window of each window, or none (kRoute)
   __nv_bfloat16* out;
   Geometry g;
   int B, heads;
   int q_quads;                  // ceil(nw_max / 512): 512-query units per window
+  FastDiv f_qq, f_nw, f_heads;  // by q_quads, n_windows, heads
   int total_units;
   int n_slots;
   float scale_log2;
@@ -728,9 +768,14 @@ struct __align__(64) PairParams {
   int stall;                    // test hook: the MMA issuer first waits on a barrier nothing arrives on
 };
 
+// Query tiles are double-buffered: the units a CTA pair runs alternate between
+// two sets of two tiles, so the next unit's queries load while the current one
+// runs.  When a unit is done, its set's tile i holds the bf16 output rows of
+// tile i on their way to the TMA stores, and is refilled only after those
+// stores have read it.
 struct PairCtl {
-  uint64_t q_full[2];           // leader: both CTAs' Q tile i landed
-  uint64_t q_empty[2];          // both: Q tile i may be overwritten
+  uint64_t q_full[2][2];        // leader: both CTAs' Q tile i of set s landed
+  uint64_t q_free[2][2];        // each CTA: its Q tile i of set s may be refilled
   uint64_t kv_full[kPairMaxSlots];   // leader: both halves of a ring slot landed
   uint64_t kv_empty[kPairMaxSlots];  // both: ring slot may be overwritten
   uint64_t s_full[2];           // both: S_i in TMEM
@@ -758,11 +803,11 @@ __device__ __forceinline__ bool pair_wait(uint64_t* bar, uint32_t parity, PairCt
 // A pair unit: up to 512 queries; tile i of CTA c holds slots q0 + 256 i + 128 c + [0, 128).
 template <bool kMem, bool kRoute>
 __device__ __forceinline__ bool decode_pair_unit(const PairParams& p, int u, Unit& U) {
-  const int qp = u % p.q_quads;
-  const int r = u / p.q_quads;
-  const int win_id = r % p.g.n_windows;
-  const int bh = r / p.g.n_windows;
-  U.b = bh / p.heads;
+  const int r = fdiv(u, p.f_qq);
+  const int qp = u - r * p.q_quads;
+  const int bh = fdiv(r, p.f_nw);
+  const int win_id = r - bh * p.g.n_windows;
+  U.b = fdiv(bh, p.f_heads);
   U.h = bh - U.b * p.heads;
   window_of(p.g, win_id, U.m, U.e);
   U.n_valid = U.e[0] * U.e[1] * U.e[2];
@@ -781,11 +826,6 @@ __device__ __forceinline__ bool decode_pair_unit(const PairParams& p, int u, Uni
   return true;
 }
 
-__device__ __forceinline__ int pair_row(const PairParams& p, const Unit& U, int slot) {
-  if (slot >= U.n_valid) slot = U.n_valid - 1;
-  return (U.b * p.g.N + slot_token(p.g, U.m, U.e, slot)) * p.heads + U.h;
-}
-
 // Keys of tile j used by the MMAs: all 128, or the valid keys rounded up to 32
 // for the last tile (each CTA then holds half of them).
 template <bool kMem, bool kRoute>
@@ -802,8 +842,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                                              ~static_cast<uintptr_t>(1023));
   constexpr int kQBytes = kTile * 128 * 2;
   const int n_slots = p.n_slots;
-  uint8_t* sQ = smem;                                   // two own query tiles
-  uint8_t* sRing = sQ + 2 * kQBytes;                    // K/V half tiles
+  uint8_t* sQ = smem;                                   // two sets of two own query tiles
+  uint8_t* sRing = sQ + 4 * kQBytes;                    // K/V half tiles
   PairCtl* ctl = reinterpret_cast<PairCtl*>(sRing + n_slots * kPairHalfTileBytes);
 
   const int warp = threadIdx.x >> 5;
@@ -814,9 +854,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   const int n_clusters = gridDim.x >> 1;
 
   if (threadIdx.x == 0) {
+    for (int s = 0; s < 2; ++s)
+      for (int i = 0; i < 2; ++i) {
+        mbar_init(&ctl->q_full[s][i], 1);
+        mbar_init(&ctl->q_free[s][i], 4);
+      }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&ctl->q_full[i], 1);
-      mbar_init(&ctl->q_empty[i], 1);
       mbar_init(&ctl->s_full[i], 1);
       mbar_init(&ctl->p_full[i], 8);
       mbar_init(&ctl->o_final[i], 1);
@@ -834,6 +877,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     prefetch_tensormap(&p.tq);
     prefetch_tensormap(&p.tk);
     prefetch_tensormap(&p.tv);
+    prefetch_tensormap(&p.to);
   }
   if (warp == kPairMmaWarp) {
     tmem_alloc_pair(&ctl->tmem_base, kTmemCols);
@@ -849,8 +893,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     // Gathers of every tile are spread over the producer warps' lanes (see
     // `gathers`).  Loads land in this CTA and are counted on the leader's barriers.
     const int pw = warp - kPairProducer0;
-    uint32_t q_use[2] = {0, 0};
+    // Q buffer b = 2 * set + tile: bit b of q_par is the parity of the loads
+    // into it so far, bit b of q_loaded is set once it has been loaded
+    uint32_t q_par = 0, q_loaded = 0;
     uint32_t ld = 0;
+    uint32_t lu = 0;                           // units of this CTA pair so far
     bool ok = true;
     // `count` gathers numbered 0..count-1 cover slots slot0 + [0, 4 * count / nblk):
     // gather n covers row group n / nblk (slots slot0 + 4 (n / nblk) + [0, 4)) and
@@ -878,20 +925,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     for (int u = cluster_id; ok && u < p.total_units; u += n_clusters) {
       Unit U;
       if (!decode_pair_unit<kMem, kRoute>(p, u, U)) continue;
+      const int set = lu & 1;
+      ++lu;
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
         if (i == 1 && !U.has_q1) break;
-        if (q_use[i] > 0) {
-          ok = __all_sync(0xffffffffu, pair_wait(&ctl->q_empty[i], (q_use[i] - 1) & 1, ctl,
+        const uint32_t b = 2 * set + i;
+        if ((q_loaded >> b) & 1) {
+          ok = __all_sync(0xffffffffu, pair_wait(&ctl->q_free[set][i], ((q_par >> b) & 1) ^ 1, ctl,
                                                  p.timeout_ns, false));
           if (!ok) break;
         }
-        const uint32_t bar = map_to_rank(smem_u32(&ctl->q_full[i]), 0);
-        if (leader && pw == 0 && elect_one()) mbar_arrive_expect_tx(&ctl->q_full[i], 2 * kQBytes);
+        const uint32_t bar = map_to_rank(smem_u32(&ctl->q_full[set][i]), 0);
+        if (leader && pw == 0 && elect_one()) mbar_arrive_expect_tx(&ctl->q_full[set][i], 2 * kQBytes);
         __syncwarp();
-        gathers(U, &p.tq, bar, sQ + i * kQBytes, U.q0 + i * 2 * kTile + static_cast<int>(rank) * kTile, 64, 2,
-                kTile * 128, 0, 0);
-        ++q_use[i];
+        gathers(U, &p.tq, bar, sQ + (2 * set + i) * kQBytes,
+                U.q0 + i * 2 * kTile + static_cast<int>(rank) * kTile, 64, 2, kTile * 128, 0, 0);
+        q_par ^= 1u << b;
+        q_loaded |= 1u << b;
       }
       for (int j = 0; ok && j < U.nkv; ++j) {
         const int ns = pair_ns<kMem, kRoute>(U, j);
@@ -926,24 +977,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     // Drain: in the leader, every load of either CTA is counted on these
     // barriers; the final cluster barrier keeps the peer alive until then.
     if (leader) {
-      for (int i = 0; i < 2; ++i)
-        if (q_use[i] > 0) mbar_wait_bounded(&ctl->q_full[i], (q_use[i] - 1) & 1, drain_ns(p.timeout_ns));
+      for (int b = 0; b < 4; ++b)
+        if ((q_loaded >> b) & 1)
+          mbar_wait_bounded(&ctl->q_full[b >> 1][b & 1], ((q_par >> b) & 1) ^ 1, drain_ns(p.timeout_ns));
       for (uint32_t x = (ld > static_cast<uint32_t>(n_slots) ? ld - n_slots : 0); x < ld; ++x)
         mbar_wait_bounded(&ctl->kv_full[x % n_slots], (x / n_slots) & 1, drain_ns(p.timeout_ns));
     }
   } else if (warp == kPairMmaWarp) {
     // ================================================================ MMA issuer (leader)
     if (leader && lane == 0) {
-      const uint32_t q_addr0 = smem_u32(sQ);
       const uint32_t ring_addr = smem_u32(sRing);
       const uint32_t idesc_pv = idesc_bf16_f32(256, 128, 0, 1);
-      uint32_t q_use[2] = {0, 0};
+      uint32_t q_par = 0;     // bit 2 * set + tile: parity of the uses of that Q buffer so far
       uint32_t p_use[2] = {0, 0};
       uint32_t ld = 0;
+      uint32_t lu = 0;
       bool ok = !p.stall || pair_wait(&ctl->never, 0, ctl, p.timeout_ns, false);
-      auto issue_qk = [&](int i, uint32_t k_addr, int ns) {
+      auto issue_qk = [&](uint32_t q_addr, int i, uint32_t k_addr, int ns) {
         const uint32_t idesc = idesc_bf16_f32(256, ns, 0, 0);
-        const uint32_t q_addr = q_addr0 + i * kQBytes;
         for (int kk = 0; kk < 8; ++kk) {
           umma_ss_pair(tmem + (i ? kColS1 : kColS0),
                        smem_desc_sw128(q_addr + (kk >> 2) * (kTile * 128) + (kk & 3) * 32, 16, 1024),
@@ -961,10 +1012,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       for (int u = cluster_id; ok && u < p.total_units; u += n_clusters) {
         Unit U;
         if (!decode_pair_unit<kMem, kRoute>(p, u, U)) continue;
+        const int set = lu & 1;
+        ++lu;
+        const uint32_t q_addr[2] = {smem_u32(sQ + (2 * set) * kQBytes), smem_u32(sQ + (2 * set + 1) * kQBytes)};
         const int nq = U.has_q1 ? 2 : 1;
 #pragma unroll
         for (int i = 0; i < 2; ++i)
-          if (ok && i < nq) ok = pair_wait(&ctl->q_full[i], q_use[i] & 1, ctl, p.timeout_ns, false);
+          if (ok && i < nq)
+            ok = pair_wait(&ctl->q_full[set][i], (q_par >> (2 * set + i)) & 1, ctl, p.timeout_ns, false);
         if (!ok) break;
         int slot_k = ld % n_slots;
         ok = pair_wait(&ctl->kv_full[slot_k], (ld / n_slots) & 1, ctl, p.timeout_ns, false);
@@ -974,9 +1029,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
           if (i >= nq) break;
-          issue_qk(i, ring_addr + slot_k * kPairHalfTileBytes, pair_ns<kMem, kRoute>(U, 0));
+          issue_qk(q_addr[i], i, ring_addr + slot_k * kPairHalfTileBytes, pair_ns<kMem, kRoute>(U, 0));
           umma_commit_pair(&ctl->s_full[i], 3);
-          if (U.nkv == 1) umma_commit_pair(&ctl->q_empty[i], 3);
         }
         umma_commit_pair(&ctl->kv_empty[slot_k], 3);
         for (int j = 0; j < U.nkv; ++j) {
@@ -1004,16 +1058,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                 ++ld;
                 tc_fence_after();
               }
-              issue_qk(i, ring_addr + slot_k * kPairHalfTileBytes, pair_ns<kMem, kRoute>(U, j + 1));
+              issue_qk(q_addr[i], i, ring_addr + slot_k * kPairHalfTileBytes, pair_ns<kMem, kRoute>(U, j + 1));
               umma_commit_pair(&ctl->s_full[i], 3);
-              if (j + 1 == U.nkv - 1) umma_commit_pair(&ctl->q_empty[i], 3);
               if (i == nq - 1) umma_commit_pair(&ctl->kv_empty[slot_k], 3);
             }
           }
           if (!ok) break;
         }
-        ++q_use[0];
-        if (nq == 2) ++q_use[1];
+        q_par ^= (nq == 2 ? 3u : 1u) << (2 * set);
       }
       umma_commit_pair(&ctl->drained, 1);
       mbar_wait_bounded(&ctl->drained, 0, drain_ns(p.timeout_ns));
@@ -1029,11 +1081,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     const uint32_t p_full_leader = map_to_rank(smem_u32(&ctl->p_full[wg]), 0);
     const float sl2 = p.scale_log2;
     uint32_t s_use = 0, of_use = 0;
+    uint32_t lu = 0;
+    int pending = -1;   // set whose tile wg holds output rows the TMA stores may still be reading
+    // Hands tile wg of set `pending` back to the producers once this warp's
+    // stores have read it.
+    auto release = [&]() {
+      if (pending >= 0) {
+        bulk_wait_group_read0();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl->q_free[pending][wg]);
+        pending = -1;
+      }
+    };
     bool ok = true;
     for (int u = cluster_id; ok && u < p.total_units; u += n_clusters) {
       Unit U;
       if (!decode_pair_unit<kMem, kRoute>(p, u, U)) continue;
-      if (wg == 1 && !U.has_q1) continue;
+      const int set = lu & 1;
+      ++lu;
+      if (wg == 1 && !U.has_q1) {
+        release();
+        continue;
+      }
       float m_run = -INFINITY;
       float l_run = 0.0f;
       for (int j = 0; j < U.nkv; ++j) {
@@ -1059,34 +1128,69 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(p_full_leader);
+        if (j == 0) release();   // the previous unit's stores read their tile long ago
       }
       if (!ok) break;
       ok = __all_sync(0xffffffffu, pair_wait(&ctl->o_final[wg], of_use & 1, ctl, p.timeout_ns, false));
       if (!ok) break;
       ++of_use;
       tc_fence_after();
-      const int slot = U.q0 + wg * 2 * kTile + static_cast<int>(rank) * kTile + row;
-      const bool valid = slot < U.n_valid;
-      __nv_bfloat16* dst = nullptr;
-      if (valid) dst = p.out + static_cast<size_t>(pair_row(p, U, slot)) * 128;
+      // the unit's window geometry, decoded again rather than held in registers
+      // through the key loop
+      decode_pair_unit<kMem, kRoute>(p, u, U);
+      // ---- epilogue: O / l in bf16 into this tile's (now unused) query buffer,
+      // laid out as a load through the same tensor map leaves rows (row r at
+      // r * 128 in each 64-column block, 16-byte chunk c at position c ^ (r & 7)),
+      // then tile::scatter4 stores put each group of four rows at the rows its
+      // queries came from (the inverse roll) while this warp moves on.
+      uint8_t* stage = sQ + (2 * set + wg) * kQBytes;
       const float inv_l = 1.0f / l_run;
+      uint32_t ra[32], rb[32];
+      tmem_ld32(tO, ra);
+      tmem_wait_ld();
+      tmem_tie(ra);
+#pragma unroll
       for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tO + c * 32, r);
-        tmem_wait_ld();
-        uint32_t pk[16];
+        uint32_t(&cur)[32] = (c & 1) ? rb : ra;
+        uint32_t(&nxt)[32] = (c & 1) ? ra : rb;
+        if (c < 3) tmem_ld32(tO + (c + 1) * 32, nxt);
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * inv_l, __uint_as_float(r[2 * i + 1]) * inv_l);
-        if (valid) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+        for (int v4 = 0; v4 < 4; ++v4) {
+          const int q = 4 * c + v4;   // 16-byte chunk of the 256-byte row
+          uint32_t pk[4];
 #pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4)
-            d4[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+          for (int e = 0; e < 4; ++e)
+            pk[e] = pack_bf16x2(__uint_as_float(cur[8 * v4 + 2 * e]) * inv_l,
+                                __uint_as_float(cur[8 * v4 + 2 * e + 1]) * inv_l);
+          st_shared_v4(stage + (q >> 3) * (kTile * 128) + row * 128 + (((q & 7) ^ (row & 7)) << 4), pk[0], pk[1],
+                       pk[2], pk[3]);
+        }
+        if (c < 3) {
+          tmem_wait_ld();
+          tmem_tie(nxt);
         }
       }
-      tc_fence_before();
+      tc_fence_before();   // O_i reads are ordered before the next unit's P V (via p_full)
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane < 16) {
+        // lane l stores rows rbase .. rbase + 3 of this warp's 32, column block l & 1;
+        // groups made only of padding rows (past the window's tokens) are not stored,
+        // and padding rows inside a group repeat the window's last query, whose own
+        // result they equal
+        const int rbase = (warp & 3) * 32 + 4 * (lane >> 1);
+        const int slot0 = U.q0 + wg * 2 * kTile + static_cast<int>(rank) * kTile + rbase;
+        if (slot0 < U.n_valid) {
+          int rr[4];
+          unit_rows4(p.g, U, p.heads, slot0, rr);
+          tma_scatter4(&p.to, stage + (lane & 1) * (kTile * 128) + rbase * 128, 64 * (lane & 1), rr[0], rr[1],
+                       rr[2], rr[3]);
+        }
+        bulk_commit_group();
+      }
+      pending = set;
     }
+    bulk_wait_group0();   // every store of this warp is complete before the CTA exits
   }
 
   tc_fence_before();
@@ -1312,13 +1416,18 @@ static size_t smem_bytes_for(int d) {
 static int g_sm_count[kMaxDevices];
 static int g_pair_clusters[kMaxDevices];   // co-resident CTA pairs of the pair kernel
 
+// Dynamic shared memory a CTA may use on sm_100 (227 KB).
+constexpr size_t kMaxDynSmem = 232448;
+
 static int pair_slots() {
-  int slots = (200 * 1024 - 2 * kTile * 128 * 2) / kPairHalfTileBytes;
+  // K/V ring: as many half tiles as fit next to the four query tiles (two sets)
+  const size_t fixed = 1024 + static_cast<size_t>(4 * kTile * 128 * 2) + sizeof(PairCtl);
+  const int slots = static_cast<int>((kMaxDynSmem - fixed) / kPairHalfTileBytes);
   return slots > kPairMaxSlots ? kPairMaxSlots : slots;
 }
 
 static size_t pair_smem_bytes() {
-  return 1024 + static_cast<size_t>(2 * kTile * 128 * 2) +
+  return 1024 + static_cast<size_t>(4 * kTile * 128 * 2) +
          static_cast<size_t>(pair_slots()) * kPairHalfTileBytes + sizeof(PairCtl);
 }
 
@@ -1469,7 +1578,7 @@ static int launch_fwd(const void* q, const void* k, const void* v, const int* ro
     PairParams pp;
     memset(&pp, 0, sizeof(pp));
     if (encode_rows(&pp.tq, q, rows, d) || encode_rows(&pp.tk, k, rows, d) ||
-        encode_rows(&pp.tv, v, rows, d))
+        encode_rows(&pp.tv, v, rows, d) || encode_rows(&pp.to, out, rows, d))
       return BASA_ERR_CUDA;
     if (E > 0 && (encode_rows(&pp.tkx, kx, xrows, d) || encode_rows(&pp.tvx, vx, xrows, d)))
       return BASA_ERR_CUDA;
@@ -1480,6 +1589,9 @@ static int launch_fwd(const void* q, const void* k, const void* v, const int* ro
     pp.B = B;
     pp.heads = heads;
     pp.q_quads = static_cast<int>(q_quads);
+    pp.f_qq = make_fastdiv(pp.q_quads);
+    pp.f_nw = make_fastdiv(g.n_windows);
+    pp.f_heads = make_fastdiv(heads);
     pp.total_units = static_cast<int>(punits);
     pp.n_slots = pair_slots();
     pp.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
@@ -1507,6 +1619,9 @@ static int launch_fwd(const void* q, const void* k, const void* v, const int* ro
   p.heads = heads;
   p.d = d;
   p.q_pairs = static_cast<int>(q_pairs);
+  p.f_qp = make_fastdiv(p.q_pairs);
+  p.f_nw = make_fastdiv(g.n_windows);
+  p.f_heads = make_fastdiv(heads);
   p.total_units = static_cast<int>(units);
   p.n_slots = slots_for(d);
   p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);

@@ -44,6 +44,13 @@ def _run_gpu(q, k, v, grid, win, shift, scale):
     return out
 
 
+def _full_compare_inputs(q, k, v, B, heads, d, grid, win, shift, scale):
+    T, H, W = grid
+    out = _run_gpu(q, k, v, grid, win, shift, scale).float().cpu().numpy()
+    ref = oracle.swattn_fwd(q, k, v, B, heads, T, H, W, d, win, shift, scale)
+    return _check(out, ref, f"grid={grid} win={win} shift={shift} d={d}")
+
+
 def _full_compare(B, heads, d, grid, win, shift, scale=None, seed=0, dist="normal"):
     T, H, W = grid
     q, k, v = make_custom(B, heads, d, T, H, W, seed, dist=dist)
@@ -108,6 +115,24 @@ def test_full_attention_mode_tiny():
 def test_sharp_softmax_exercises_rescaling():
     # scale 1 with d = 128 gives logits of std ~11: the running max moves a lot.
     _full_compare(1, 2, 128, (1, 24, 24), (1, 12, 12), (0, 6, 6), scale=1.0, seed=21)
+
+
+@pytest.mark.parametrize("d", [128, 64])
+def test_logits_jump_by_hundreds_between_key_tiles(d):
+    # keys of the window's later key tiles are planted as large multiples of
+    # their query, so the row maximum grows by far more than fp32 exponents
+    # span (~2^130) from one key tile to the next: the running maximum must
+    # move (O rescaled) without any intermediate overflow
+    grid, win, shift = (1, 24, 24), (1, 24, 12), (0, 0, 5)     # 288-token windows: tiles 0-127, 128-255, 256-287
+    q, k, v = make_custom(1, 2, d, *grid, seed=40 + d)
+    tos, cnt = oracle.index_map(*grid, win, shift)
+    rng = np.random.default_rng(d)
+    for wid in range(tos.shape[0]):
+        for slot in (150, 200, 270):
+            tok = int(tos[wid, slot])
+            src = int(tos[wid, int(rng.integers(0, 128))])     # a query of the first tile
+            k[0, tok] = (q[0, src].float() * (4.0 if slot < 256 else 8.0)).to(torch.bfloat16)
+    _full_compare_inputs(q, k, v, 1, 2, d, grid, win, shift, 1.0 / math.sqrt(d))
 
 
 def test_uniform_inputs():
