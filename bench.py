@@ -24,6 +24,7 @@ The last line printed on stdout by rank 0 is the JSON result.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import datetime
 import hashlib
 import json
@@ -451,6 +452,13 @@ def run_native(args):
     peaks, peak_src = load_peaks()
     peak_tflops = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     wl = BY_NAME[args.workload]
+    if args.heads:
+        # a smaller case of the same workload (profiling captures): fewer heads,
+        # the same grid, windows and shifts
+        wl = dataclasses.replace(wl, heads=args.heads)
+    if args.full_attention:
+        # the same kernel run as full attention (window = whole grid, no shift)
+        wl = dataclasses.replace(wl, win=wl.grid, shifts=((0, 0, 0),))
     stream = torch.cuda.current_stream(device)
     q, k, v = make_qkv(wl, device=device, seed=wl.seed + 1000 * rank)
     out = torch.empty_like(q)
@@ -640,18 +648,22 @@ def run_native(args):
                                    f"threads, CPU {cpu_model()}")}
 
     traffic_rec = load_traffic()
+    # the recorded traffic is that of the default headline configuration
+    custom = bool(args.heads) or args.full_attention or args.workload != HEADLINE
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": wl_config(wl, {"parallelism": f"replicas x{world}" if world > 1 else "single GPU"}),
+        "config": wl_config(wl, {"parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                                 **({"mode": "full attention"} if args.full_attention else {})}),
         "frac_of_peak": achieved / peak_tflops,
         "peak_source": f"{peak_src} bf16 dense burst ({peak_tflops:.1f} TFLOP/s)",
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_tflops,
                      "unit": "TFLOP/s", "frac": achieved / peak_tflops,
-                     "traffic": traffic_rec["dram_bytes_per_launch"] if traffic_rec else None,
-                     "kernel": KERNEL_NAME, "flops_per_launch": f_layer,
+                     "traffic": traffic_rec["dram_bytes_per_launch"] if traffic_rec and not custom else None,
+                     "kernel": KERNEL_NAME if wl.d == 128 else "swattn_fwd_kernel",
+                     "flops_per_launch": f_layer,
                      "ms_per_launch": ms_launch,
                      "peak_kind": f"{peak_src} burst"},
         "cpu_baseline": cpu_base,
@@ -693,6 +705,10 @@ def main():
                          "(the `text_memory` key)")
     ap.add_argument("--schedule-layers", type=int, default=8,
                     help="also time an L-layer stack under the interleaved shift schedule (0: off)")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="override the workload's head count (a smaller case of it, for profiling captures)")
+    ap.add_argument("--full-attention", action="store_true",
+                    help="run the step in full-attention mode (window = grid, shift 0), for profiling captures")
     ap.add_argument("--workload", default=HEADLINE,
                     help="workload name from shifted_window_attention_swattn_b200.inputs "
                          "(profiling runs of a smaller case; the default is the headline)")
