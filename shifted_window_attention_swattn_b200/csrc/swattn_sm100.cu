@@ -993,21 +993,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       uint32_t ld = 0;
       uint32_t lu = 0;
       bool ok = !p.stall || pair_wait(&ctl->never, 0, ctl, p.timeout_ns, false);
+      // Descriptors of the K = 16 slices are the tile's base descriptor plus the
+      // slice's byte offset / 16 (the start-address field; shared-memory
+      // addresses are 16-byte multiples far below 2^18, so the field never
+      // carries into its neighbours).
       auto issue_qk = [&](uint32_t q_addr, int i, uint32_t k_addr, int ns) {
         const uint32_t idesc = idesc_bf16_f32(256, ns, 0, 0);
-        for (int kk = 0; kk < 8; ++kk) {
-          umma_ss_pair(tmem + (i ? kColS1 : kColS0),
-                       smem_desc_sw128(q_addr + (kk >> 2) * (kTile * 128) + (kk & 3) * 32, 16, 1024),
-                       smem_desc_sw128(k_addr + (kk >> 2) * (64 * 128) + (kk & 3) * 32, 16, 1024),
-                       idesc, kk > 0 ? 1u : 0u);
-        }
+        const uint64_t qd = smem_desc_sw128(q_addr, 16, 1024), kd = smem_desc_sw128(k_addr, 16, 1024);
+        const uint32_t tS = tmem + (i ? kColS1 : kColS0);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ss_pair(tS, qd + (((kk >> 2) * (kTile * 128) + (kk & 3) * 32) >> 4),
+                       kd + (((kk >> 2) * (64 * 128) + (kk & 3) * 32) >> 4), idesc, kk > 0 ? 1u : 0u);
       };
       auto issue_pv = [&](int i, uint32_t v_addr, int ns, bool acc) {
         const uint32_t tS = tmem + (i ? kColS1 : kColS0);
         const uint32_t tO = tmem + (i ? kColO1 : kColO0);
-        for (int kk = 0; kk < ns / 16; ++kk)
-          umma_ts_pair(tO, tS + kk * 8, smem_desc_sw128(v_addr + kk * 2048, kTile * 128, 1024),
-                       idesc_pv, (acc || kk > 0) ? 1u : 0u);
+        const uint64_t vd = smem_desc_sw128(v_addr, kTile * 128, 1024);
+        if (ns == kTile) {
+#pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk)
+            umma_ts_pair(tO, tS + kk * 8, vd + kk * (2048 >> 4), idesc_pv, (acc || kk > 0) ? 1u : 0u);
+        } else {
+          for (int kk = 0; kk < ns / 16; ++kk)
+            umma_ts_pair(tO, tS + kk * 8, vd + kk * (2048 >> 4), idesc_pv, (acc || kk > 0) ? 1u : 0u);
+        }
       };
       for (int u = cluster_id; ok && u < p.total_units; u += n_clusters) {
         Unit U;
