@@ -439,11 +439,21 @@ __device__ __forceinline__ float softmax_row_step(uint32_t tS, int kv_valid, flo
 // S_i (+)= Q_i K^T over the head dimension: d/16 MMAs of M=128, N=n_s, K=16.
 __device__ __forceinline__ void issue_qk(uint32_t tmem_s, uint32_t q_addr, uint32_t k_addr, int d,
                                          int n_s) {
+  // Descriptors of the K = 16 slices are the tile's base descriptor plus the
+  // slice's byte offset / 16 in the start-address field (shared-memory
+  // addresses stay below 2^18, so the field never carries).
   const uint32_t idesc = idesc_bf16_f32(128, n_s, 0, 0);
-  for (int kk = 0; kk < d / 16; ++kk) {
-    const uint32_t off = (kk >> 2) * (kTile * 128) + (kk & 3) * 32;
-    umma_ss(tmem_s, smem_desc_sw128(q_addr + off, 16, 1024), smem_desc_sw128(k_addr + off, 16, 1024),
-            idesc, kk > 0 ? 1u : 0u);
+  const uint64_t qd = smem_desc_sw128(q_addr, 16, 1024), kd = smem_desc_sw128(k_addr, 16, 1024);
+  if (d == 64) {
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+      umma_ss(tmem_s, qd + ((kk * 32) >> 4), kd + ((kk * 32) >> 4), idesc, kk > 0 ? 1u : 0u);
+  } else {
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      const uint32_t off = ((kk >> 2) * (kTile * 128) + (kk & 3) * 32) >> 4;
+      umma_ss(tmem_s, qd + off, kd + off, idesc, kk > 0 ? 1u : 0u);
+    }
   }
 }
 
@@ -451,10 +461,16 @@ __device__ __forceinline__ void issue_qk(uint32_t tmem_s, uint32_t q_addr, uint3
 __device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint32_t v_addr, int d,
                                          int kv_valid, bool accumulate) {
   const uint32_t idesc = idesc_bf16_f32(128, d, 0, 1);
+  const uint64_t vd = smem_desc_sw128(v_addr, kTile * 128, 1024);
   const int ksteps = (kv_valid + 15) >> 4;
-  for (int kk = 0; kk < ksteps; ++kk)
-    umma_ts(tmem_o, tmem_p + kk * 8, smem_desc_sw128(v_addr + kk * 2048, kTile * 128, 1024), idesc,
-            (accumulate || kk > 0) ? 1u : 0u);
+  if (ksteps == kTile / 16) {
+#pragma unroll
+    for (int kk = 0; kk < kTile / 16; ++kk)
+      umma_ts(tmem_o, tmem_p + kk * 8, vd + kk * (2048 >> 4), idesc, (accumulate || kk > 0) ? 1u : 0u);
+  } else {
+    for (int kk = 0; kk < ksteps; ++kk)
+      umma_ts(tmem_o, tmem_p + kk * 8, vd + kk * (2048 >> 4), idesc, (accumulate || kk > 0) ? 1u : 0u);
+  }
 }
 
 template <bool kMem, bool kRoute>
@@ -514,6 +530,8 @@ __global__ void __launch_bounds__(kThreads, 1) swattn_fwd_kernel(const __grid_co
     const uint32_t half_bytes = tile_bytes / kProducers;
     uint32_t q_use[2] = {0, 0};
     uint32_t ld = 0;          // loads issued into the ring
+    int fill_slot = 0;        // ld % n_slots and ld / n_slots, kept incrementally
+    uint32_t fill_use = 0;
     bool ok = true;
     // seg: the segment the tile comes from (0 window, 1 routed window, 2 extra
     // segment); slot0 counts that segment's tokens.
@@ -545,8 +563,12 @@ __global__ void __launch_bounds__(kThreads, 1) swattn_fwd_kernel(const __grid_co
       }
       for (int j = 0; ok && j < U.nkv; ++j) {
         for (int kv = 0; kv < 2; ++kv) {
-          const int slot = ld % n_slots;
-          const uint32_t use = ld / n_slots;
+          const int slot = fill_slot;
+          const uint32_t use = fill_use;
+          if (++fill_slot == n_slots) {
+            fill_slot = 0;
+            ++fill_use;
+          }
           if (use > 0) {
             ok = __all_sync(0xffffffffu,
                             wait_or_abort(&ctl->kv_empty[slot], (use - 1) & 1, ctl, p.timeout_ns));
@@ -575,7 +597,18 @@ __global__ void __launch_bounds__(kThreads, 1) swattn_fwd_kernel(const __grid_co
       const uint32_t tO[2] = {tmem + kColO0, tmem + kColO1};
       uint32_t q_use[2] = {0, 0};
       uint32_t p_use[2] = {0, 0};
-      uint32_t ld = 0;        // ring tiles consumed
+      // Ring position of the next K/V tile to consume and the parity of its
+      // fill, kept incrementally (no division between two MMA batches).
+      int kv_slot = 0;
+      uint32_t kv_phase = 0;
+      auto take = [&](int& slot, uint32_t& phase) {
+        slot = kv_slot;
+        phase = kv_phase;
+        if (++kv_slot == n_slots) {
+          kv_slot = 0;
+          kv_phase ^= 1u;
+        }
+      };
       bool ok = !p.stall || wait_or_abort(&ctl->never, 0, ctl, p.timeout_ns);
       for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
         Unit U;
@@ -586,10 +619,11 @@ __global__ void __launch_bounds__(kThreads, 1) swattn_fwd_kernel(const __grid_co
           if (ok && i < nq) ok = wait_or_abort(&ctl->q_full[i], q_use[i] & 1, ctl, p.timeout_ns);
         if (!ok) break;
         // K_0 -> S_i(0)
-        int slot_k = ld % n_slots;
-        ok = wait_or_abort(&ctl->kv_full[slot_k], (ld / n_slots) & 1, ctl, p.timeout_ns);
+        int slot_k;
+        uint32_t phase_k;
+        take(slot_k, phase_k);
+        ok = wait_or_abort(&ctl->kv_full[slot_k], phase_k, ctl, p.timeout_ns);
         if (!ok) break;
-        ++ld;
         tc_fence_after();
         {
           const int n_s = (kv_valid_of<kMem, kRoute>(U, 0) + 15) & ~15;
@@ -603,12 +637,14 @@ __global__ void __launch_bounds__(kThreads, 1) swattn_fwd_kernel(const __grid_co
           umma_commit(&ctl->kv_empty[slot_k]);
         }
         for (int j = 0; j < U.nkv; ++j) {
-          const int slot_v = ld % n_slots;
-          ok = wait_or_abort(&ctl->kv_full[slot_v], (ld / n_slots) & 1, ctl, p.timeout_ns);
+          int slot_v;
+          uint32_t phase_v;
+          take(slot_v, phase_v);
+          ok = wait_or_abort(&ctl->kv_full[slot_v], phase_v, ctl, p.timeout_ns);
           if (!ok) break;
-          ++ld;
           const bool more = j + 1 < U.nkv;
           const int kvv = kv_valid_of<kMem, kRoute>(U, j);
+          const int n_s = more ? (kv_valid_of<kMem, kRoute>(U, j + 1) + 15) & ~15 : 0;
 #pragma unroll
           for (int i = 0; i < 2; ++i) {
             if (i >= nq) break;
@@ -617,21 +653,23 @@ __global__ void __launch_bounds__(kThreads, 1) swattn_fwd_kernel(const __grid_co
             ++p_use[i];
             tc_fence_after();
             issue_pv(tO[i], tS[i], ring_addr + slot_v * tile_bytes, d, kvv, j > 0);
-            if (!more) umma_commit(&ctl->o_final[i]);
-            if (i == nq - 1) umma_commit(&ctl->kv_empty[slot_v]);
+            if (more && i == 0) {
+              // K of the next step: waited for here, after this tile's P V
+              take(slot_k, phase_k);
+              ok = wait_or_abort(&ctl->kv_full[slot_k], phase_k, ctl, p.timeout_ns);
+              if (!ok) break;
+              tc_fence_after();
+            }
             if (more) {
-              if (i == 0) {
-                slot_k = ld % n_slots;
-                ok = wait_or_abort(&ctl->kv_full[slot_k], (ld / n_slots) & 1, ctl, p.timeout_ns);
-                if (!ok) break;
-                ++ld;
-                tc_fence_after();
-              }
-              const int n_s = (kv_valid_of<kMem, kRoute>(U, j + 1) + 15) & ~15;
               issue_qk(tS[i], q_addr[i], ring_addr + slot_k * tile_bytes, d, n_s);
               umma_commit(&ctl->s_full[i]);
               if (j + 1 == U.nkv - 1) umma_commit(&ctl->q_empty[i]);
-              if (i == nq - 1) umma_commit(&ctl->kv_empty[slot_k]);
+            } else {
+              umma_commit(&ctl->o_final[i]);
+            }
+            if (i == nq - 1) {
+              umma_commit(&ctl->kv_empty[slot_v]);
+              if (more) umma_commit(&ctl->kv_empty[slot_k]);
             }
           }
           if (!ok) break;
@@ -897,6 +935,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     // into it so far, bit b of q_loaded is set once it has been loaded
     uint32_t q_par = 0, q_loaded = 0;
     uint32_t ld = 0;
+    int fill_slot = 0;                         // ld % n_slots and ld / n_slots, kept incrementally
+    uint32_t fill_use = 0;
     uint32_t lu = 0;                           // units of this CTA pair so far
     bool ok = true;
     // `count` gathers numbered 0..count-1 cover slots slot0 + [0, 4 * count / nblk):
@@ -948,8 +988,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         const int ns = pair_ns<kMem, kRoute>(U, j);
         const int half = ns >> 1;
         for (int kv = 0; kv < 2; ++kv) {
-          const int slot = ld % n_slots;
-          const uint32_t use = ld / n_slots;
+          const int slot = fill_slot;
+          const uint32_t use = fill_use;
+          if (++fill_slot == n_slots) {
+            fill_slot = 0;
+            ++fill_use;
+          }
           if (use > 0) {
             ok = __all_sync(0xffffffffu, pair_wait(&ctl->kv_empty[slot], (use - 1) & 1, ctl,
                                                    p.timeout_ns, false));
@@ -990,7 +1034,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       const uint32_t idesc_pv = idesc_bf16_f32(256, 128, 0, 1);
       uint32_t q_par = 0;     // bit 2 * set + tile: parity of the uses of that Q buffer so far
       uint32_t p_use[2] = {0, 0};
-      uint32_t ld = 0;
+      // Ring position of the next K/V tile to consume and the parity of its
+      // fill, kept incrementally: this thread's code between two MMA batches
+      // runs on the critical path, so no division or remainder appears there.
+      int kv_slot = 0;
+      uint32_t kv_phase = 0;
+      auto take = [&](int& slot, uint32_t& phase) {
+        slot = kv_slot;
+        phase = kv_phase;
+        if (++kv_slot == n_slots) {
+          kv_slot = 0;
+          kv_phase ^= 1u;
+        }
+      };
       uint32_t lu = 0;
       bool ok = !p.stall || pair_wait(&ctl->never, 0, ctl, p.timeout_ns, false);
       // Descriptors of the K = 16 slices are the tile's base descriptor plus the
@@ -1031,10 +1087,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           if (ok && i < nq)
             ok = pair_wait(&ctl->q_full[set][i], (q_par >> (2 * set + i)) & 1, ctl, p.timeout_ns, false);
         if (!ok) break;
-        int slot_k = ld % n_slots;
-        ok = pair_wait(&ctl->kv_full[slot_k], (ld / n_slots) & 1, ctl, p.timeout_ns, false);
+        int slot_k;
+        uint32_t phase_k;
+        take(slot_k, phase_k);
+        ok = pair_wait(&ctl->kv_full[slot_k], phase_k, ctl, p.timeout_ns, false);
         if (!ok) break;
-        ++ld;
         tc_fence_after();
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
@@ -1044,12 +1101,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         }
         umma_commit_pair(&ctl->kv_empty[slot_k], 3);
         for (int j = 0; j < U.nkv; ++j) {
-          const int slot_v = ld % n_slots;
-          ok = pair_wait(&ctl->kv_full[slot_v], (ld / n_slots) & 1, ctl, p.timeout_ns, false);
+          // V of this step and K of the next: both are waited for here, before
+          // the first P is, so that a tile's P V and Q K^T batches follow each
+          // other with nothing in between
+          int slot_v;
+          uint32_t phase_v;
+          take(slot_v, phase_v);
+          ok = pair_wait(&ctl->kv_full[slot_v], phase_v, ctl, p.timeout_ns, false);
           if (!ok) break;
-          ++ld;
           const bool more = j + 1 < U.nkv;
+          if (more) {
+            take(slot_k, phase_k);
+            ok = pair_wait(&ctl->kv_full[slot_k], phase_k, ctl, p.timeout_ns, false);
+            if (!ok) break;
+          }
           const int ns = pair_ns<kMem, kRoute>(U, j);
+          const int ns_next = more ? pair_ns<kMem, kRoute>(U, j + 1) : 0;
 #pragma unroll
           for (int i = 0; i < 2; ++i) {
             if (i >= nq) break;
@@ -1058,19 +1125,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             ++p_use[i];
             tc_fence_after();
             issue_pv(i, ring_addr + slot_v * kPairHalfTileBytes, ns, j > 0);
-            if (!more) umma_commit_pair(&ctl->o_final[i], 3);
-            if (i == nq - 1) umma_commit_pair(&ctl->kv_empty[slot_v], 3);
             if (more) {
-              if (i == 0) {
-                slot_k = ld % n_slots;
-                ok = pair_wait(&ctl->kv_full[slot_k], (ld / n_slots) & 1, ctl, p.timeout_ns, false);
-                if (!ok) break;
-                ++ld;
-                tc_fence_after();
-              }
-              issue_qk(q_addr[i], i, ring_addr + slot_k * kPairHalfTileBytes, pair_ns<kMem, kRoute>(U, j + 1));
+              issue_qk(q_addr[i], i, ring_addr + slot_k * kPairHalfTileBytes, ns_next);
               umma_commit_pair(&ctl->s_full[i], 3);
-              if (i == nq - 1) umma_commit_pair(&ctl->kv_empty[slot_k], 3);
+            } else {
+              umma_commit_pair(&ctl->o_final[i], 3);
+            }
+            if (i == nq - 1) {
+              umma_commit_pair(&ctl->kv_empty[slot_v], 3);
+              if (more) umma_commit_pair(&ctl->kv_empty[slot_k], 3);
             }
           }
           if (!ok) break;
