@@ -31,6 +31,22 @@ def test_strip_c_comments_keeps_escaped_quotes_in_literals():
     assert b.strip_c_comments(src) == 'const char* s = "a \\" // still inside"; int x;'
 
 
+def test_comment_stripping_keeps_code_and_literals():
+    b = _bench()
+    src = 'int a = 1; // note\n/* block\n comment */ const char* s = "x//y/*z*/";\nchar c = \'"\';  float b;'
+    assert b.strip_c_comments(src) == 'int a = 1; const char* s = "x//y/*z*/"; char c = \'"\'; float b;'
+
+
+def test_kernel_hash_ignores_comments_but_not_code():
+    b = _bench()
+    base = {rel: "int f() { return 1; }\n" for rel in b.KERNEL_SOURCES}
+    commented = {rel: "// header\nint f() { /* one */ return 1; }   \n" for rel in b.KERNEL_SOURCES}
+    changed = {rel: "int f() { return 2; }\n" for rel in b.KERNEL_SOURCES}
+    h = b.kernel_source_hash(base.__getitem__)
+    assert h == b.kernel_source_hash(commented.__getitem__)
+    assert h != b.kernel_source_hash(changed.__getitem__)
+
+
 def _hash_with(b, edit):
     texts = {}
     for rel in b.KERNEL_SOURCES:
